@@ -206,7 +206,7 @@ static long double pmean(const double *m, int64_t K, double p)
 {
     if (isinf(p)) {
         double mx = 0.0;
-        for (int64_t k = 0; k < K; ++k) if (m[k] > mx) mx = m[k];
+        for (int64_t k = 0; k < K; ++k) if (isnan(m[k]) || m[k] > mx) mx = m[k];
         return mx;
     }
     long double s = 0.0L;
@@ -219,7 +219,10 @@ double oracle_pmean(const double *m, int64_t K, double p) { return (double)pmean
 /* ------------------------------------------- one row of MX quantisation */
 
 /* Quantise one row y[0..D) (fp32 values) to E4M3 codes + E8M0 scales [RC][F8].
-   rounding: 0 = nearest-even, 1 = stochastic with Philox words. */
+   rounding: 0 = nearest-even, 1 = stochastic with Philox words.
+   A block holding an infinity or a NaN (outside the method's contract) gets
+   the NaN scale 0xFF and the positive NaN code 0x7F for every element: the
+   sign of a NaN made by 0 * inf differs between platforms, so none is kept. */
 static void mx_quantise_row(const float *y, int64_t D, uint8_t *q, uint8_t *scales,
                             int rounding, uint64_t seed, uint64_t row)
 {
@@ -237,7 +240,7 @@ static void mx_quantise_row(const float *y, int64_t D, uint8_t *q, uint8_t *scal
         scales[k] = e8m0_code(e);
         for (int i = 0; i < ORACLE_BLOCK; ++i) {
             int64_t col = k * ORACLE_BLOCK + i;
-            if (e == 128) { q[col] = (signbit(yb[i]) ? 0x80 : 0) | 0x7F; continue; }
+            if (e == 128) { q[col] = 0x7F; continue; }           /* non-finite block: NaN code */
             float inv_scale = ldexpf(1.0f, -e);           /* 2^-e, exact in fp32 */
             float v = yb[i] * inv_scale;                  /* fp32 product, as the kernel */
             if (rounding == 0) q[col] = oracle_e4m3_rne(v);
@@ -283,7 +286,7 @@ int oracle_mxnorm_fwd(const uint16_t *x, int64_t ld_x, const uint16_t *gamma,
             double mk = 0.0;
             for (int j = 0; j < ORACLE_BLOCK; ++j) {
                 double v = fabs((double)bf16_to_f32(xr[k * ORACLE_BLOCK + j]));
-                if (v > mk) mk = v;
+                if (isnan(v) || v > mk) mk = v;   /* a NaN, once seen, stays the max */
             }
             m[k] = mk;
         }

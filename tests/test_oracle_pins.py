@@ -294,6 +294,23 @@ def test_zero_row_and_zero_block():
     assert s[1, 0] == 0 and np.all(q[1, :32] == 0)
 
 
+def test_nonfinite_inputs_mark_blocks_nan():
+    """Out of contract, but defined: NaN/inf give scale 0xFF and code 0x7F per block."""
+    D = 128
+    x = torch.ones(3, D, dtype=torch.bfloat16)
+    x[0, 5] = float("nan")
+    x[1, 70] = float("inf")
+    x[2, 33] = -float("inf")
+    q, s, G = oracle.mxnorm_fwd(x, None, 2.0)
+    assert math.isnan(G[0]) and np.all(s[0] == 0xFF) and np.all(q[0] == 0x7F)
+    # an infinite row statistic: s = 1/inf = 0, so only the inf element's block is NaN
+    assert math.isinf(G[1]) and list(s[1]) == [0, 0, 0xFF, 0]
+    assert np.all(q[1, 64:96] == 0x7F) and np.all(q[1, :64] == 0)
+    assert list(s[2]) == [0, 0xFF, 0, 0] and np.all(q[2, 32:64] == 0x7F)
+    qc, sc = oracle.mxfp8_cast(x)
+    assert list(sc[1]) == [0x77, 0x77, 0xFF, 0x77] and np.all(qc[1, 64:96] == 0x7F)
+
+
 def test_scales_fit_and_are_minimal():
     """Every block fits under its scale, and would not under half of it."""
     D = 2048
