@@ -1,0 +1,436 @@
+"""MXNorm forward benchmark on B200: GB/s and fraction of HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-extras]
+
+One step = one MXNorm forward (block absmax -> p-mean G -> 1/G * gamma ->
+E8M0 scales + E4M3 codes, one kernel) over one batch of the workload, default
+x bf16 [8192 x 4096] N(0,1) with 1% outlier channels x50, gamma = 1 + 0.1 N,
+p = 2, nearest-even, row-major scales.  `value` is whole-job GB/s of algorithmic
+bytes (read x 2 B/elem, write codes 1 B/elem and scales 1/32 B/elem, gamma and
+G) with inputs resident in HBM; steps rotate over a pool of input/output sets
+larger than 3x the L2, so no step reads another's data from L2.
+
+Rank 0 prints one JSON line.  N > 1 runs one process per GPU (torchrun);
+every rank processes its own batch (weak scaling, no collective on the data
+path) and the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MXNorm fwd GB/s & % HBM peak at d=4096, vs RMSNorm+MXCast two-pass"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama8b_8192x4096_outliers_p2")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the two-pass comparator, e2e and CPU baseline legs")
+    ap.add_argument("--soak-s", type=float, default=0.5,
+                    help="untimed back-to-back steps before timing, so clocks settle under load")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def workload_cfg(name):
+    from normalisation_row_bf16_b200 import synthetic
+    w = dict(synthetic.WORKLOADS[name])
+    w.setdefault("p", 2.0)
+    return w
+
+
+def algorithmic_bytes(T, D):
+    # read x (2 B/elem), write E4M3 codes (1 B/elem) and E8M0 scales (1 per 32),
+    # read gamma (2 B/column), write G (4 B/row)
+    return T * D * 2 + T * D + T * (D // 32) + 2 * D + 4 * T
+
+
+def two_pass_bytes(T, D):
+    # RMSNorm: read x, write y (bf16); MXCast: read y, write codes + scales; gamma
+    return T * D * 2 * 2 + T * D * 2 + T * D + T * (D // 32) + 2 * D
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "normalisation_row_bf16_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"mxnorm_fwd_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    try:
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.rows = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", gpu_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        power = [float(r[3]) for r in self.rows if r[3].replace(".", "").isdigit()]
+        reasons = sorted({self.NAMES[i] for r in self.rows for i in range(4) if r[5 + i] == "Active"})
+        # samples under load: the upper half by power draw
+        loaded = sm
+        if power and len(power) == len(sm):
+            cut = statistics.median(power)
+            loaded = [s for s, p in zip(sm, power) if p >= cut] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(self.rows),
+                "power_w_max": max(power) if power else None}
+
+
+# --------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from normalisation_row_bf16_b200 import build as nbuild
+    from normalisation_row_bf16_b200 import ops, synthetic
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        nbuild.build()
+    if world > 1:
+        dist.barrier()
+    ops.lib()
+    w = workload_cfg(args.workload)
+    T, D, p = w["T"], w["D"], w["p"]
+    nbytes = algorithmic_bytes(T, D)
+    set_bytes = T * D * 2 + T * D + T * (D // 32) + 4 * T
+    n_sets = max(2, math.ceil(3 * L2_BYTES / set_bytes))
+
+    x0 = synthetic.activations(T, D, w["kind"], seed=rank, device=dev)
+    g = synthetic.gamma(D, seed=rank, device=dev)
+    xs = [x0] + [x0.clone() for _ in range(n_sets - 1)]
+    outs = [(torch.empty(T, D, dtype=torch.uint8, device=dev),
+             torch.empty(T, D // 32, dtype=torch.uint8, device=dev),
+             torch.empty(T, dtype=torch.float32, device=dev)) for _ in range(n_sets)]
+
+    def step(i):
+        q, s, G = outs[i % n_sets]
+        ops.mxnorm_fwd(xs[i % n_sets], g, p, q=q, scales=s, G=G)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}") if rank == 0 else None
+
+    for i in range(args.warmup):
+        step(i)
+    # untimed soak so that the sampled clocks reflect the loaded state
+    barrier()
+    t_end = time.time() + args.soak_s
+    i = 0
+    while time.time() < t_end:
+        for _ in range(50):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    t0.record()
+    for i in range(K):
+        ev_s[i].record()
+        step(i)
+        ev_e[i].record()
+    t1.record()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    region_ms = t0.elapsed_time(t1)
+    kern_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
+    status = ops.device_status()
+    if status != ops.MXN_OK:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    times = torch.tensor([region_ms, statistics.mean(kern_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    region_ms, mean_kern_ms = float(times[0]), float(times[1])
+    ms_per_step = region_ms / K
+    value = world * nbytes / (ms_per_step * 1e-3) / 1e9
+
+    extras = {}
+    if not args.no_extras:
+        extras = run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step)
+
+    if rank != 0:
+        return None
+    peaks, peak_src = measured_peaks()
+    achieved = nbytes / (mean_kern_ms * 1e-3) / 1e9
+    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {
+            "workload": args.workload, "T": T, "D": D, "block": 32, "p": p, "rounding": "rne",
+            "gamma": True, "scale_layout": "rowmajor", "x": w["kind"],
+            "l2": f"inputs rotate over {n_sets} sets of {set_bytes / 2**20:.0f} MiB "
+                  f"({n_sets * set_bytes / 2**20:.0f} MiB > 3x the 126 MB L2)",
+            "parallelism": f"replicas x{world}: rows sharded by rank, no collective",
+            "clock_soak_s": args.soak_s,
+        },
+        "tokens_per_s": round(world * T / (ms_per_step * 1e-3), 1),
+        "pct_hbm_peak": round(100.0 * value / (world * peak), 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(args.workload),
+                     "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json hbm_gbs' if peak_src == 'measured' else 'recipe fallback'})",
+                     "algorithmic_bytes_per_launch": nbytes,
+                     "kernel": "row_fwd_kernel<MXNorm>", "mean_launch_ms": round(mean_kern_ms, 6)},
+        "gpu_launches": K,
+        "clocks": clocks,
+    }
+    line.update(extras)
+    return line
+
+
+def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
+    """Two-pass comparator, end-to-end through host buffers, CPU oracle."""
+    import torch
+    import torch.distributed as dist
+    from normalisation_row_bf16_b200 import ops
+
+    T, D, p = w["T"], w["D"], w["p"]
+    out = {}
+    # two-pass RMSNorm -> bf16 -> MXCast, same rotation
+    n2 = max(2, math.ceil(3 * L2_BYTES / (T * D * 5)))
+    tmp = [(torch.empty(T, D, dtype=torch.bfloat16, device=dev),
+            torch.empty(T, D, dtype=torch.uint8, device=dev),
+            torch.empty(T, D // 32, dtype=torch.uint8, device=dev)) for _ in range(n2)]
+    xs2 = [xs[i % n_sets] for i in range(n2)]
+    K2 = args.steps
+
+    def step2(i):
+        y, q, s = tmp[i % n2]
+        ops.rmsnorm_then_mxcast(xs2[i % n2], g, 1e-5, y_tmp=y, q=q, scales=s)
+
+    for i in range(args.warmup):
+        step2(i)
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(K2):
+        step2(i)
+    t1.record()
+    barrier()
+    tp = torch.tensor([t0.elapsed_time(t1) / K2], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tp, op=dist.ReduceOp.MAX)
+    tp_ms = float(tp[0])
+    out["two_pass"] = {"ms_per_step": round(tp_ms, 6),
+                       "GBps_own_bytes": round(world * two_pass_bytes(T, D) / (tp_ms * 1e-3) / 1e9, 1),
+                       "kernels_per_step": 2}
+    out["speedup_vs_two_pass"] = round(tp_ms / ms_per_step, 3)
+    del tmp
+
+    # end to end through the C ABI with pinned host buffers
+    xh = xs[0].cpu().pin_memory()
+    qh = torch.empty(T, D, dtype=torch.uint8).pin_memory()
+    sh = torch.empty(T, D // 32, dtype=torch.uint8).pin_memory()
+    Gh = torch.empty(T, dtype=torch.float32).pin_memory()
+    xd = torch.empty_like(xs[0])
+    qd = torch.empty(T, D, dtype=torch.uint8, device=dev)
+    sd = torch.empty(T, D // 32, dtype=torch.uint8, device=dev)
+    Gd = torch.empty(T, dtype=torch.float32, device=dev)
+
+    def step_e2e():
+        xd.copy_(xh, non_blocking=True)
+        ops.mxnorm_fwd(xd, g, p, q=qd, scales=sd, G=Gd)
+        qh.copy_(qd, non_blocking=True)
+        sh.copy_(sd, non_blocking=True)
+        Gh.copy_(Gd, non_blocking=True)
+
+    Ke = min(args.steps, 100)
+    for _ in range(3):
+        step_e2e()
+    barrier()
+    t0.record()
+    for _ in range(Ke):
+        step_e2e()
+    t1.record()
+    barrier()
+    te = torch.tensor([t0.elapsed_time(t1) / Ke], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    te_ms = float(te[0])
+    out["e2e"] = {"value": round(world * algorithmic_bytes(T, D) / (te_ms * 1e-3) / 1e9, 2),
+                  "unit": "GB/s", "h2d_bytes_per_step": T * D * 2,
+                  "d2h_bytes_per_step": T * D + T * (D // 32) + 4 * T,
+                  "steps": Ke, "ms_per_step": round(te_ms, 4)}
+
+    # CPU oracle on the host cores: rank 0, one GPU only
+    if rank == 0 and world == 1:
+        import oracle
+        x_cpu = xs[0].cpu()
+        g_cpu = g.cpu()
+        oracle.mxnorm_fwd(x_cpu[:64], g_cpu, p)             # load + warm
+        t = time.time()
+        oracle.mxnorm_fwd(x_cpu, g_cpu, p)
+        dt = time.time() - t
+        out["cpu_baseline"] = {"value": round(algorithmic_bytes(T, D) / dt / 1e9, 3), "unit": "GB/s",
+                               "cores": oracle.num_threads(), "kind": "oracle",
+                               "sample": f"all {T} rows of the workload, once ({dt:.2f} s)"}
+    return out
+
+
+# ---------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    import torch
+    import oracle
+    from normalisation_row_bf16_b200 import synthetic
+
+    w = workload_cfg(args.workload)
+    T, D, p = w["T"], w["D"], w["p"]
+    x = synthetic.activations(T, D, w["kind"], seed=0)
+    g = synthetic.gamma(D, seed=0)
+    # size each step's sample so that warm-up + steps take about a minute
+    probe = min(T, 256)
+    t = time.time()
+    oracle.mxnorm_fwd(x[:probe], g, p)
+    per_row = (time.time() - t) / probe
+    total = args.steps + args.warmup
+    rows = int(max(1, min(T, 60.0 / max(total, 1) / max(per_row, 1e-9))))
+    xs = x[:rows].contiguous()
+    for _ in range(args.warmup):
+        oracle.mxnorm_fwd(xs, g, p)
+    t = time.time()
+    for _ in range(args.steps):
+        oracle.mxnorm_fwd(xs, g, p)
+    dt = (time.time() - t) / max(args.steps, 1)
+    value = algorithmic_bytes(rows, D) / dt / 1e9
+    cores = oracle.num_threads()
+    sample = f"rows 0..{rows - 1} of the {T}-row workload per step"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "T": T, "D": D, "block": 32, "p": p, "rounding": "rne",
+                   "gamma": True, "scale_layout": "rowmajor", "x": w["kind"]},
+        "cpu_baseline": {"kind": "oracle", "value": round(value, 4), "unit": "GB/s", "cores": cores,
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    import datetime
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,193 @@
+/*
+ * mxnorm.h -- C ABI of the B200 (sm_100a) MXNorm library, libmxnorm_b200.so.
+ *
+ * MXNorm (gist.science, "MXNorm: Reusing MXFP block scales for efficient
+ * tensor normalisation", technical summary section 2.1) replaces RMSNorm ahead
+ * of an MX-quantised linear layer.  For each row of a bf16 activation it takes
+ * the absolute maximum m_k of every block of B = 32 consecutive elements,
+ * estimates the row's RMS as their generalised p-mean
+ *     G = ((1/K) sum_k m_k^p)^(1/p),   K = D / 32,
+ * normalises the row by 1/G (and a gain gamma), and writes the result as
+ * MXFP8: one E4M3 code per element plus one E8M0 power-of-two scale per block
+ * of 32, in a single pass over HBM.
+ *
+ * Conventions shared by every entry point
+ *  - Device pointers unless stated.  The caller owns all memory; the library
+ *    never allocates device memory and keeps no pointer after returning.
+ *  - Calls are asynchronous and ordered on the CUDA stream `stream`
+ *    (a cudaStream_t; NULL means the legacy default stream).  They launch on
+ *    the device that is current on the calling thread.
+ *  - Tensors are row-major.  T = rows (tokens), D = row length (hidden size),
+ *    D a multiple of 32, 32 <= D <= MXN_MAX_D.  ld_x = distance in elements
+ *    between consecutive rows of x (ld_x >= D, a multiple of 8).  Every other
+ *    tensor is dense (its row stride is its row length).
+ *  - Every device pointer must be 16-byte aligned.
+ *  - Return value: MXN_OK (0) on success, a negative mxn_status otherwise.  On
+ *    error nothing is launched (MXN_ERR_ARG / MXN_ERR_UNSUPPORTED) or the launch
+ *    failed (MXN_ERR_CUDA); mxnorm_last_error() then describes the cause.
+ *    No entry point traps or aborts.
+ *  - E4M3 codes follow the OCP FP8 E4M3 encoding (bias 7, no infinities, NaN =
+ *    S.1111.111, largest finite 448), as "FP8 Formats for Deep Learning" (cited
+ *    on the "Recipes for Pre-training LLMs with MXFP8" page) defines it.  E8M0
+ *    scale codes c stand for 2^(c - 127); 0xFF is NaN.
+ *  - Scale rule ("Recipes for Pre-training LLMs with MXFP8", abstract, read as
+ *    "round the scale up so that no element saturates"): for a block whose
+ *    absmax is a, the scale is 2^e with e the smallest integer in [-127, 127]
+ *    such that a <= 448 * 2^e.  A block holding NaN or infinity gets scale
+ *    0xFF and code 0x7F for every element.
+ */
+#ifndef MXNORM_B200_H
+#define MXNORM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Largest supported row length. */
+#define MXN_MAX_D 32768
+
+/* Status codes. */
+enum mxn_status {
+    MXN_OK = 0,
+    MXN_ERR_ARG = -1,          /* invalid argument: shape, alignment, null, p */
+    MXN_ERR_UNSUPPORTED = -2,  /* valid but not supported here (D > MXN_MAX_D, ...) */
+    MXN_ERR_CUDA = -3,         /* a CUDA call or kernel launch failed */
+    MXN_ERR_TIMEOUT = -4       /* a kernel gave up a bounded wait (see mxnorm_device_status) */
+};
+
+/* Rounding of the E4M3 element cast. */
+enum mxn_rounding {
+    MXN_ROUND_RNE = 0,  /* nearest, ties to even, saturating to +-448 */
+    /* Stochastic rounding (aibr.jp article on stochastic rounding with BF16 and
+       Adam, section 3): a value between two neighbouring E4M3 values lo < hi
+       becomes hi with probability (|v| - lo) / (hi - lo), so its expectation is
+       v.  The draw is word (idx & 3) of Philox4x32-10 (Salmon et al., SC'11)
+       with key = (seed low 32 bits, seed high 32 bits) and counter =
+       (idx >> 2 low 32 bits, idx >> 2 high 32 bits, 0, 0), idx = row * D + col
+       (independent of ld_x); hi is taken iff word < frac * 2^32, exactly. */
+    MXN_ROUND_SR = 1
+};
+
+/* Layout of the E8M0 scales. */
+enum mxn_scale_layout {
+    /* scales[row * K + k], K = D / 32: one byte per block, row-major. */
+    MXN_SCALES_ROWMAJOR = 0,
+    /* The layout tcgen05 block-scaled MMA consumes (128 x 4 tiles, K-major):
+       rows padded to a multiple of 128 and K to a multiple of 4; the byte of
+       (row, k) is at ((row / 128) * (Kp / 4) + k / 4) * 512 + (row % 32) * 16
+       + ((row % 128) / 32) * 4 + (k % 4), Kp = K rounded up to 4.  Padding
+       bytes are not written. */
+    MXN_SCALES_MMA = 1
+};
+
+/* Bytes the scales of a [T, D] tensor occupy in the given layout; 0 if the
+   arguments are invalid. */
+size_t mxnorm_scales_bytes(int64_t T, int64_t D, int layout);
+
+/*
+ * MXNorm forward (MXNorm page, technical summary section 2.1; gain as in
+ * section 2.3).  For every row r of x:
+ *   m_k   = max over block k of |x|                          (exact)
+ *   G_r   = ((1/K) sum_k m_k^p)^(1/p) in fp32; p = +inf gives max_k m_k
+ *   s     = fl32(1 / G_r)  (s = 0 when G_r = 0)
+ *   y_j   = fl32(x_j * s), then y_j = fl32(y_j * gamma_j) if gamma != NULL
+ *   per block: scale 2^e from max |y| (rule above); code_j = E4M3(fl32(y_j * 2^-e))
+ * x       bf16 [T, ld_x] (first D columns used)
+ * gamma   bf16 [D] or NULL (NULL when the gain is folded into the next
+ *         layer's weight, section 2.3)
+ * q       uint8 [T, D] E4M3 codes (written)
+ * scales  uint8, mxnorm_scales_bytes(T, D, scale_layout) bytes (written)
+ * G_out   fp32 [T] (written) or NULL; the backward pass takes it.
+ * p       > 0 (INFINITY allowed); 2 is the default the page settles on
+ *         (section 3.1: p = 1 was unstable at 8B parameters).
+ * rounding  enum mxn_rounding; seed is used only by MXN_ROUND_SR.
+ * G_out agrees with the exact p-mean to about 1e-6 relative (fp32 reduction).
+ */
+int mxnorm_fwd(const void* x, const void* gamma, void* q, void* scales, float* G_out,
+               int64_t T, int64_t D, int64_t ld_x, float p, int rounding, uint64_t seed,
+               int scale_layout, void* stream);
+
+/*
+ * MX quantisation of x itself (MXCast; MXNorm page, technical summary section
+ * 1.2): y = x, then the per-block scale and code of mxnorm_fwd.
+ * Same argument meanings as mxnorm_fwd.
+ */
+int mxfp8_cast(const void* x, void* q, void* scales, int64_t T, int64_t D, int64_t ld_x,
+               int rounding, uint64_t seed, int scale_layout, void* stream);
+
+/*
+ * RMSNorm (MXNorm page, sections 1.1-1.2, the layer MXNorm replaces):
+ *   y = bf16( fl32(x * 1/sqrt(mean(x^2) + eps)) * gamma ), fp32 arithmetic.
+ * x bf16 [T, ld_x]; gamma bf16 [D] or NULL; y bf16 [T, D] (written).
+ */
+int rmsnorm_bf16(const void* x, const void* gamma, void* y, int64_t T, int64_t D, int64_t ld_x,
+                 float eps, void* stream);
+
+/*
+ * The two-pass comparator of MXNorm (section 1.2, RMSNorm and MXCast as
+ * separate steps): rmsnorm_bf16 into y_tmp, then mxfp8_cast of y_tmp with
+ * nearest-even rounding.  y_tmp bf16 [T, D] is caller-owned scratch and holds
+ * the RMSNorm output afterwards.  scales in scale_layout.
+ */
+int rmsnorm_then_mxcast(const void* x, const void* gamma, float eps, void* y_tmp, void* q,
+                        void* scales, int64_t T, int64_t D, int64_t ld_x, int scale_layout,
+                        void* stream);
+
+/*
+ * MXNorm backward (MXNorm page, technical summary section 2.3: the RMSNorm
+ * gradient reused as a straight-through estimator; the cast is taken as the
+ * identity).  With g = gamma * dy (gamma = 1 when NULL), per row:
+ *   dx     = ( g - x * (x . g) / (x . x) ) / G
+ *   dgamma = sum over rows of dy * x / G
+ * (the exact gradient of x -> x * gamma / (c * rms(x)) when G = c * rms(x)).
+ * A row with G = 0 or x = 0 gets dx = 0 and adds nothing to dgamma.
+ * x, dy   bf16 [T, D] dense; gamma bf16 [D] or NULL; G fp32 [T] from mxnorm_fwd.
+ * dx      bf16 [T, D] (written; fp32 arithmetic, one rounding).
+ * dgamma  bf16 [D] (written) or NULL; must be NULL when gamma is NULL.
+ *         Deterministic: partial sums in a fixed order, no atomics.
+ * workspace  device scratch of at least mxnorm_bwd_workspace_size(T, D)
+ *         bytes (fp32 partial sums), 16-byte aligned; may be NULL when dgamma
+ *         is NULL.  Contents on entry are ignored.
+ */
+int mxnorm_bwd(const void* x, const void* dy, const void* gamma, const float* G, void* dx,
+               void* dgamma, int64_t T, int64_t D, void* workspace, size_t workspace_bytes,
+               void* stream);
+
+/* Scratch bytes mxnorm_bwd needs for (T, D) on the current device. */
+size_t mxnorm_bwd_workspace_size(int64_t T, int64_t D);
+
+/* Message for the last error on the calling thread ("" if none).  The string
+   stays valid until the thread's next call into the library. */
+const char* mxnorm_last_error(void);
+
+/*
+ * Waits for `stream`, then reads and clears the current device's status word.
+ * Kernels that wait on a barrier bound each wait (about a second); a wait that
+ * gives up records itself there and the kernel returns early, its outputs then
+ * being incomplete.  Returns MXN_OK, MXN_ERR_TIMEOUT, or MXN_ERR_CUDA.
+ */
+int mxnorm_device_status(void* stream);
+
+/*
+ * Launch tuning for the row kernels (all four ops): consumer threads per CTA
+ * (128, 256 or 512), pipeline stages (2..16) and CTAs per SM (1..8); 0 keeps
+ * the library's choice.  Process-wide; not thread-safe against concurrent
+ * launches.  Returns MXN_ERR_ARG for out-of-range values.
+ */
+int mxnorm_set_tuning(int consumer_threads, int stages, int ctas_per_sm);
+
+/*
+ * Test hook: the next `count` entry-point calls on this thread fail with
+ * MXN_ERR_CUDA before launching (host-side fault injection; nothing runs on
+ * the GPU).  count = 0 clears it.
+ */
+void mxnorm_debug_fail_next(int count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXNORM_B200_H */

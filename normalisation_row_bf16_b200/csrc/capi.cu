@@ -1,0 +1,451 @@
+// capi.cu -- the C ABI declared in include/mxnorm.h: argument checks, launch
+// planning and error reporting around the row kernels.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+
+#include "mxnorm.h"
+#include "row_bwd.cuh"
+#include "row_fwd.cuh"
+
+// Device status word: kernels record a bounded wait that gave up here.
+__device__ unsigned g_mxn_status;
+
+namespace {
+
+using namespace mxn;
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxBwdD = 16384;
+
+thread_local std::string t_err;
+thread_local int t_fail_next = 0;
+
+struct Tuning {
+  int consumer_threads = 0, stages = 0, ctas_per_sm = 0;
+} g_tuning;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MXN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+  int sms = 0;
+  unsigned* status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// SM count and the status word's device address for the current device,
+// looked up once per device.
+int device_info(DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MXN_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.sms == 0) {
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_mxn_status);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    d.status = static_cast<unsigned*>(p);
+    d.sms = sms;
+  }
+  *out = d;
+  return MXN_OK;
+}
+
+int injected() {
+  if (t_fail_next > 0) {
+    --t_fail_next;
+    return fail(MXN_ERR_CUDA, "injected failure (mxnorm_debug_fail_next)");
+  }
+  return MXN_OK;
+}
+
+int next_pow2(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+int ilog2(int v) {
+  int l = 0;
+  while ((1 << l) < v) ++l;
+  return l;
+}
+
+// Launch plan for a row kernel: rows split into row blocks of rps rows, one
+// consumer thread per 32-element block (bpt blocks when K > 512), a ring of
+// `stages` shared-memory stages, a persistent grid of SMs x resident CTAs.
+struct Plan {
+  RowCfg C;
+  const void* kernel = nullptr;
+  int bpt = 1;
+  int threads = 0;
+  size_t smem = 0;
+  int grid = 0;
+};
+
+using KernelPicker = const void* (*)(int bpt, int nct);
+
+// Resident CTAs per SM of (kernel, threads, dynamic shared memory) on the
+// current device.  The first use of a combination sets the kernel's dynamic
+// shared-memory limit and queries the occupancy; later launches reuse both,
+// so a launch costs one map lookup on the host.
+std::map<std::tuple<int, const void*, int, size_t>, int> g_occ;
+std::mutex g_occ_mu;
+
+int occupancy(const void* kernel, int threads, size_t smem, int* occ) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const auto key = std::make_tuple(dev, kernel, threads, smem);
+  {
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    auto it = g_occ.find(key);
+    if (it != g_occ.end()) {
+      *occ = it->second;
+      return MXN_OK;
+    }
+  }
+  // Raise the kernel's dynamic shared-memory limit to the device maximum, so
+  // that no plan can shrink it below what another cached plan launches with.
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(smem optin)");
+  if (smem > (size_t)optin) return fail(MXN_ERR_UNSUPPORTED, "%zu bytes of shared memory > %d", smem, optin);
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  int n = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+  std::lock_guard<std::mutex> lk(g_occ_mu);
+  g_occ[key] = n;
+  *occ = n;
+  return MXN_OK;
+}
+
+int plan_rows(int64_t T, int D, int64_t ld_x, int n_inputs, KernelPicker pick, int sms, Plan* P) {
+  RowCfg& C = P->C;
+  C.T = T;
+  C.ld_x = ld_x;
+  C.D = D;
+  C.K = D / kBlock;
+  P->bpt = C.K > kMaxConsumerThreads ? 2 : 1;
+  C.tpr = next_pow2((C.K + P->bpt - 1) / P->bpt);
+  C.log2_tpr = ilog2(C.tpr);
+  int nct = g_tuning.consumer_threads ? g_tuning.consumer_threads : 128;
+  if (nct < C.tpr) nct = C.tpr;
+  if (P->bpt == 2) nct = kMaxConsumerThreads;
+  C.rps = nct / C.tpr;
+  C.n_cwarps = nct / 32;
+  C.row_bytes = 2u * (uint32_t)D;
+  C.stage_bytes = (uint32_t)C.rps * C.row_bytes * (uint32_t)n_inputs;
+  int stages = g_tuning.stages;
+  if (!stages) {
+    stages = (int)(49152u / C.stage_bytes);
+    stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
+  }
+  C.stages = stages;
+  C.n_row_blocks = (T + C.rps - 1) / C.rps;
+  const size_t red = (C.tpr > 32) ? (size_t)2 * C.rps * kRedSlots * sizeof(float2) : 0;
+  P->smem = (size_t)stages * C.stage_bytes + (size_t)2 * stages * sizeof(uint64_t) + red;
+  P->threads = nct + 32;
+  P->kernel = pick(P->bpt, nct);
+  if (!P->kernel) return fail(MXN_ERR_UNSUPPORTED, "no kernel for D = %d", D);
+  if (P->smem > 227u * 1024u)
+    return fail(MXN_ERR_UNSUPPORTED, "row of %d elements needs %zu bytes of shared memory", D, P->smem);
+  int occ = 0;
+  int rc = occupancy(P->kernel, P->threads, P->smem, &occ);
+  if (rc) return rc;
+  if (occ < 1) return fail(MXN_ERR_UNSUPPORTED, "row kernel does not fit on an SM (D = %d)", D);
+  if (g_tuning.ctas_per_sm && g_tuning.ctas_per_sm < occ) occ = g_tuning.ctas_per_sm;
+  const int64_t g = (int64_t)sms * occ;
+  P->grid = (int)(C.n_row_blocks < g ? C.n_row_blocks : g);
+  return MXN_OK;
+}
+
+int launch(const Plan& P, void* args, cudaStream_t stream) {
+  void* argv[] = {args, const_cast<RowCfg*>(&P.C)};
+  cudaError_t e = cudaLaunchKernel(P.kernel, dim3(P.grid), dim3(P.threads), argv, P.smem, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "row kernel launch");
+  return MXN_OK;
+}
+
+int check_common(const void* x, int64_t T, int64_t D, int64_t ld_x) {
+  if (!x) return fail(MXN_ERR_ARG, "x is NULL");
+  if (T < 0) return fail(MXN_ERR_ARG, "T = %lld < 0", (long long)T);
+  if (D <= 0 || D % kBlock != 0) return fail(MXN_ERR_ARG, "D = %lld is not a positive multiple of 32", (long long)D);
+  if (D > MXN_MAX_D) return fail(MXN_ERR_UNSUPPORTED, "D = %lld > %d", (long long)D, MXN_MAX_D);
+  if (ld_x < D || ld_x % 8 != 0)
+    return fail(MXN_ERR_ARG, "ld_x = %lld must be >= D and a multiple of 8", (long long)ld_x);
+  if (!aligned16(x)) return fail(MXN_ERR_ARG, "x is not 16-byte aligned");
+  return MXN_OK;
+}
+
+int check_out(const void* p, const char* name) {
+  if (!p) return fail(MXN_ERR_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(MXN_ERR_ARG, "%s is not 16-byte aligned", name);
+  return MXN_OK;
+}
+
+int check_opt(const void* p, const char* name) {
+  if (p && !aligned16(p)) return fail(MXN_ERR_ARG, "%s is not 16-byte aligned", name);
+  return MXN_OK;
+}
+
+template <int MODE, bool SR>
+const void* fwd_kernel(int bpt, int nct) {
+  if (bpt == 2) return (const void*)row_fwd_kernel<MODE, 2, 512, SR>;
+  switch (nct) {
+    case 128: return (const void*)row_fwd_kernel<MODE, 1, 128, SR>;
+    case 256: return (const void*)row_fwd_kernel<MODE, 1, 256, SR>;
+    case 512: return (const void*)row_fwd_kernel<MODE, 1, 512, SR>;
+    default: return nullptr;
+  }
+}
+
+const void* bwd_kernel(int bpt, int nct) {
+  if (bpt != 1) return nullptr;
+  switch (nct) {
+    case 128: return (const void*)row_bwd_kernel<128>;
+    case 256: return (const void*)row_bwd_kernel<256>;
+    case 512: return (const void*)row_bwd_kernel<512>;
+    default: return nullptr;
+  }
+}
+
+template <int MODE>
+int launch_fwd(const FwdArgs& A, int64_t T, int D, int64_t ld_x, cudaStream_t stream) {
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  Plan P;
+  KernelPicker pick = A.sr ? fwd_kernel<MODE, true> : fwd_kernel<MODE, false>;
+  if (MODE == kModeRMSNorm) pick = fwd_kernel<MODE, false>;
+  rc = plan_rows(T, D, ld_x, 1, pick, dev.sms, &P);
+  if (rc) return rc;
+  FwdArgs a = A;
+  a.status = dev.status;
+  return launch(P, &a, stream);
+}
+
+int pmode_of(float p) {
+  if (std::isinf(p)) return kPInf;
+  if (p == 1.0f) return kP1;
+  if (p == 2.0f) return kP2;
+  if (p == 4.0f) return kP4;
+  return kPGeneral;
+}
+
+int plan_bwd(int64_t T, int D, int sms, Plan* P) {
+  return plan_rows(T, D, D, 2, bwd_kernel, sms, P);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mxnorm_scales_bytes(int64_t T, int64_t D, int layout) {
+  if (T < 0 || D <= 0 || D % kBlock != 0) return 0;
+  const int64_t K = D / kBlock;
+  if (layout == MXN_SCALES_ROWMAJOR) return (size_t)(T * K);
+  if (layout == MXN_SCALES_MMA) return (size_t)(((T + 127) / 128) * 128 * ((K + 3) / 4) * 4);
+  return 0;
+}
+
+static int fwd_like(int mode, const void* x, const void* gamma, void* q, void* scales, float* G_out,
+                    int64_t T, int64_t D, int64_t ld_x, float p, int rounding, uint64_t seed,
+                    int scale_layout, void* stream) {
+  t_err.clear();
+  int rc = check_common(x, T, D, ld_x);
+  if (!rc) rc = check_out(q, "q");
+  if (!rc) rc = check_out(scales, "scales");
+  if (!rc) rc = check_opt(gamma, "gamma");
+  if (!rc) rc = check_opt(G_out, "G_out");
+  if (rc) return rc;
+  if (mode == kModeMXNorm && !(p > 0.0f)) return fail(MXN_ERR_ARG, "p = %g must be > 0", (double)p);
+  if (rounding != MXN_ROUND_RNE && rounding != MXN_ROUND_SR)
+    return fail(MXN_ERR_ARG, "rounding = %d", rounding);
+  if (scale_layout != MXN_SCALES_ROWMAJOR && scale_layout != MXN_SCALES_MMA)
+    return fail(MXN_ERR_ARG, "scale_layout = %d", scale_layout);
+  if ((rc = injected())) return rc;
+  if (T == 0) return MXN_OK;
+  FwdArgs A{};
+  A.x = static_cast<const uint16_t*>(x);
+  A.gamma = static_cast<const uint16_t*>(gamma);
+  A.q = static_cast<uint8_t*>(q);
+  A.scales = static_cast<uint8_t*>(scales);
+  A.G_out = G_out;
+  A.p = p;
+  A.inv_p = std::isinf(p) ? 0.0f : 1.0f / p;
+  A.pmode = pmode_of(p);
+  A.sr = rounding == MXN_ROUND_SR;
+  A.seed_lo = (uint32_t)seed;
+  A.seed_hi = (uint32_t)(seed >> 32);
+  A.scale_mma = scale_layout == MXN_SCALES_MMA;
+  A.kp4 = (int)(((D / kBlock) + 3) / 4 * 4);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return mode == kModeMXNorm ? launch_fwd<kModeMXNorm>(A, T, (int)D, ld_x, s)
+                             : launch_fwd<kModeCast>(A, T, (int)D, ld_x, s);
+}
+
+int mxnorm_fwd(const void* x, const void* gamma, void* q, void* scales, float* G_out, int64_t T,
+               int64_t D, int64_t ld_x, float p, int rounding, uint64_t seed, int scale_layout,
+               void* stream) {
+  return fwd_like(kModeMXNorm, x, gamma, q, scales, G_out, T, D, ld_x, p, rounding, seed,
+                  scale_layout, stream);
+}
+
+int mxfp8_cast(const void* x, void* q, void* scales, int64_t T, int64_t D, int64_t ld_x,
+               int rounding, uint64_t seed, int scale_layout, void* stream) {
+  return fwd_like(kModeCast, x, nullptr, q, scales, nullptr, T, D, ld_x, 1.0f, rounding, seed,
+                  scale_layout, stream);
+}
+
+int rmsnorm_bf16(const void* x, const void* gamma, void* y, int64_t T, int64_t D, int64_t ld_x,
+                 float eps, void* stream) {
+  t_err.clear();
+  int rc = check_common(x, T, D, ld_x);
+  if (!rc) rc = check_out(y, "y");
+  if (!rc) rc = check_opt(gamma, "gamma");
+  if (rc) return rc;
+  if (!(eps >= 0.0f)) return fail(MXN_ERR_ARG, "eps = %g must be >= 0", (double)eps);
+  if ((rc = injected())) return rc;
+  if (T == 0) return MXN_OK;
+  FwdArgs A{};
+  A.x = static_cast<const uint16_t*>(x);
+  A.gamma = static_cast<const uint16_t*>(gamma);
+  A.y = static_cast<uint16_t*>(y);
+  A.eps = eps;
+  return launch_fwd<kModeRMSNorm>(A, T, (int)D, ld_x, static_cast<cudaStream_t>(stream));
+}
+
+int rmsnorm_then_mxcast(const void* x, const void* gamma, float eps, void* y_tmp, void* q,
+                        void* scales, int64_t T, int64_t D, int64_t ld_x, int scale_layout,
+                        void* stream) {
+  // Every argument of both passes is checked before the first launch.
+  t_err.clear();
+  int rc = check_common(x, T, D, ld_x);
+  if (!rc) rc = check_out(y_tmp, "y_tmp");
+  if (!rc) rc = check_out(q, "q");
+  if (!rc) rc = check_out(scales, "scales");
+  if (!rc) rc = check_opt(gamma, "gamma");
+  if (rc) return rc;
+  if (!(eps >= 0.0f)) return fail(MXN_ERR_ARG, "eps = %g must be >= 0", (double)eps);
+  if (scale_layout != MXN_SCALES_ROWMAJOR && scale_layout != MXN_SCALES_MMA)
+    return fail(MXN_ERR_ARG, "scale_layout = %d", scale_layout);
+  rc = rmsnorm_bf16(x, gamma, y_tmp, T, D, ld_x, eps, stream);
+  if (rc) return rc;
+  return mxfp8_cast(y_tmp, q, scales, T, D, D, MXN_ROUND_RNE, 0, scale_layout, stream);
+}
+
+size_t mxnorm_bwd_workspace_size(int64_t T, int64_t D) {
+  if (T <= 0 || D <= 0 || D % kBlock != 0 || D > kMaxBwdD) return 0;
+  DeviceInfo dev;
+  if (device_info(&dev)) return 0;
+  Plan P;
+  if (plan_bwd(T, (int)D, dev.sms, &P)) return 0;
+  return (size_t)P.grid * P.C.rps * (size_t)D * sizeof(float);
+}
+
+int mxnorm_bwd(const void* x, const void* dy, const void* gamma, const float* G, void* dx,
+               void* dgamma, int64_t T, int64_t D, void* workspace, size_t workspace_bytes,
+               void* stream) {
+  t_err.clear();
+  int rc = check_common(x, T, D, D);
+  if (!rc) rc = check_out(dy, "dy");
+  if (!rc) rc = check_out(G, "G");
+  if (!rc) rc = check_out(dx, "dx");
+  if (!rc) rc = check_opt(gamma, "gamma");
+  if (!rc) rc = check_opt(dgamma, "dgamma");
+  if (rc) return rc;
+  if (D > kMaxBwdD) return fail(MXN_ERR_UNSUPPORTED, "mxnorm_bwd: D = %lld > %d", (long long)D, kMaxBwdD);
+  if (dgamma && !gamma) return fail(MXN_ERR_ARG, "dgamma requested without gamma");
+  if ((rc = injected())) return rc;
+  if (T == 0) return MXN_OK;
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  Plan P;
+  if ((rc = plan_bwd(T, (int)D, dev.sms, &P))) return rc;
+  const size_t need = (size_t)P.grid * P.C.rps * (size_t)D * sizeof(float);
+  if (dgamma) {
+    if (!workspace || !aligned16(workspace))
+      return fail(MXN_ERR_ARG, "workspace is NULL or not 16-byte aligned");
+    if (workspace_bytes < need)
+      return fail(MXN_ERR_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+  }
+  BwdArgs A{};
+  A.x = static_cast<const uint16_t*>(x);
+  A.dy = static_cast<const uint16_t*>(dy);
+  A.gamma = static_cast<const uint16_t*>(gamma);
+  A.G = G;
+  A.dx = static_cast<uint16_t*>(dx);
+  A.partial = dgamma ? static_cast<float*>(workspace) : nullptr;
+  A.status = dev.status;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = launch(P, &A, s))) return rc;
+  if (dgamma) {
+    dgamma_reduce_kernel<<<(unsigned)((D + 31) / 32), dim3(32, 32), 0, s>>>(
+        A.partial, (int64_t)P.grid * P.C.rps, (int)D, static_cast<uint16_t*>(dgamma));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "dgamma_reduce_kernel launch");
+  }
+  return MXN_OK;
+}
+
+const char* mxnorm_last_error(void) { return t_err.c_str(); }
+
+int mxnorm_device_status(void* stream) {
+  t_err.clear();
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_mxn_status, sizeof v);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol(status)");
+  if (v) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_mxn_status, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol(status)");
+    return fail(MXN_ERR_TIMEOUT, "a kernel gave up a bounded wait (status 0x%x)", v);
+  }
+  return MXN_OK;
+}
+
+int mxnorm_set_tuning(int consumer_threads, int stages, int ctas_per_sm) {
+  t_err.clear();
+  if (consumer_threads != 0 && consumer_threads != 128 && consumer_threads != 256 &&
+      consumer_threads != 512)
+    return fail(MXN_ERR_ARG, "consumer_threads = %d", consumer_threads);
+  if (stages != 0 && (stages < 2 || stages > 16)) return fail(MXN_ERR_ARG, "stages = %d", stages);
+  if (ctas_per_sm < 0 || ctas_per_sm > 8) return fail(MXN_ERR_ARG, "ctas_per_sm = %d", ctas_per_sm);
+  g_tuning.consumer_threads = consumer_threads;
+  g_tuning.stages = stages;
+  g_tuning.ctas_per_sm = ctas_per_sm;
+  return MXN_OK;
+}
+
+void mxnorm_debug_fail_next(int count) { t_fail_next = count > 0 ? count : 0; }
+
+}  // extern "C"

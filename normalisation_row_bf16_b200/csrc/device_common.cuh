@@ -1,0 +1,224 @@
+// device_common.cuh -- sm_100a device helpers for the MXNorm row kernels.
+//
+// Inline PTX for the bulk-copy (TMA engine) pipeline, bounded mbarrier waits,
+// and the MX element arithmetic: E8M0 scale from a block absmax, the E4M3
+// cast, Philox4x32-10 and stochastic rounding.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mxn {
+
+constexpr int kBlock = 32;                       // MX block size B
+constexpr uint64_t kWaitLimitNs = 1000000000ull; // bounded waits give up after ~1 s
+
+// Status bits recorded in the device status word.
+constexpr unsigned kStatusWaitTimeout = 1u;
+
+// ----------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+// Make the initialised barriers visible to the async (bulk-copy) proxy.
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait until the phase of `bar` with the given parity has completed, for at
+// most kWaitLimitNs.  Returns false (and records the timeout in *status) if
+// the wait gave up.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  unsigned* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(status, kStatusWaitTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// 1-D bulk copy global -> shared on the TMA engine, completing `bytes` of
+// transaction count on `bar`.  Needs 16-byte aligned addresses and a size that
+// is a multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gmem_src,
+                                              uint32_t bytes, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// L2 policy for data read exactly once: evict first.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// Streaming 16-byte global store (written once, not re-read here).
+__device__ __forceinline__ void stg128_stream(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 ldg128_nc(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// ------------------------------------------------------------- float helpers
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// max(a, |b|) propagating NaN.
+__device__ __forceinline__ float max_abs_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(fabsf(b)));
+  return d;
+}
+
+// Absolute maximum of 32 bf16 values held as 16 packed words, as fp32.  The
+// comparison runs on the magnitude bits (for non-negative floats the integer
+// order is the numeric order), so a NaN, whose magnitude bits exceed those of
+// every number, propagates.
+__device__ __forceinline__ uint32_t absmax_bits_bf16x2(const uint32_t* w, int n) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < n; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+__device__ __forceinline__ float bf16bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+// 2^n for an integer n in [-126, 127], built from its exponent field.
+__device__ __forceinline__ float exp2_int(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
+
+// ------------------------------------------------------------------ E8M0 scale
+
+// Scale exponent of a block whose absmax has fp32 bits `abits` (non-negative):
+// the smallest e in [-127, 127] with a <= 448 * 2^e.  Writing a = m * 2^E with
+// m in [1, 2), 448 = 1.75 * 2^8 gives e = E - 8 when m <= 1.75, else E - 7.
+// Zero and fp32 subnormals give -127.  Returns 128 for NaN / infinity.
+__device__ __forceinline__ int e8m0_exponent_bits(uint32_t abits) {
+  if (abits >= 0x7F800000u) return 128;
+  const int ef = (int)(abits >> 23);
+  int e = ef - 127 - 8 + ((abits & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  if (ef == 0) e = -127;
+  return max(e, -127);  // finite fp32 keeps e <= 120
+}
+
+// ------------------------------------------------------------------ E4M3 cast
+
+// Two fp32 -> two E4M3 codes, round to nearest even, saturating finite; the
+// code of `lo` in bits 0..7, of `hi` in bits 8..15.
+__device__ __forceinline__ uint32_t cvt_e4m3x2_rn(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return (uint32_t)r;
+}
+
+// ---------------------------------------------------------- Philox4x32-10
+
+// Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, SC'11): each round
+// multiplies words 0 and 2 by fixed odd constants, swaps the halves and xors
+// in the round key; the key advances by the Weyl constants between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+  constexpr uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+  constexpr uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) { k0 += W0; k1 += W1; }
+    const uint32_t hi0 = __umulhi(M0, c.x), lo0 = M0 * c.x;
+    const uint32_t hi1 = __umulhi(M1, c.z), lo1 = M1 * c.z;
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// Stochastic rounding of v (|v| <= 448, finite) onto the E4M3 grid, returned
+// as the fp32 grid value (exact) with v's sign.  lo = the grid value at or
+// below |v|, step = grid spacing there; up iff r < (|v| - lo) / step * 2^32.
+// Every intermediate is exact in fp32: lo is |v| with its low mantissa bits
+// cleared (or a multiple of 2^-9 below 2^-6), |v| - lo is exact, and the
+// scaling by 2^32 / step is a power of two; for an integer r, r < t holds iff
+// r < ceil(t), and ceil(t) < 2^32.
+__device__ __forceinline__ float sr_e4m3_grid(float v, uint32_t r) {
+  const float a = fabsf(v);
+  const uint32_t ab = __float_as_uint(a);
+  float lo, step, inv_step_2_32;
+  if (ab >= 0x3C800000u) {  // |v| >= 2^-6: 3 fraction bits kept
+    lo = __uint_as_float(ab & 0xFFF00000u);
+    const uint32_t ebits = ab & 0x7F800000u;          // 2^E
+    step = __uint_as_float(ebits - (3u << 23));       // 2^(E-3)
+    inv_step_2_32 = __uint_as_float((uint32_t)(127 + 127 + 3 + 32) * (1u << 23) - ebits);  // 2^(35-E)
+  } else {                  // subnormal range of E4M3: step 2^-9
+    lo = truncf(a * 512.0f) * (1.0f / 512.0f);
+    step = 1.0f / 512.0f;
+    inv_step_2_32 = 2199023255552.0f;                 // 2^41
+  }
+  const float t = (a - lo) * inv_step_2_32;
+  const uint32_t thr = __float2uint_ru(t);
+  const float m = (r < thr) ? lo + step : lo;
+  return copysignf(m, v);
+}
+
+}  // namespace mxn

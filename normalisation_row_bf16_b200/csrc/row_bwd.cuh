@@ -1,0 +1,218 @@
+// row_bwd.cuh -- MXNorm backward.
+//
+// gist.science, "MXNorm: Reusing MXFP block scales for efficient tensor
+// normalisation", technical summary section 2.3: the backward reuses the
+// RMSNorm gradient as a straight-through estimator (the MX cast counts as the
+// identity).  With g = gamma * dy and the forward's statistic G:
+//     dx     = ( g - x * (x . g) / (x . x) ) / G
+//     dgamma = sum over rows of dy * x / G
+// which is the exact gradient of x -> x * gamma / (c * rms(x)) at G = c * rms(x).
+//
+// Same pipeline as the forward (row_fwd.cuh): a producer thread streams the x
+// row and the dy row of each row block into a shared-memory stage with 1-D
+// bulk copies; a consumer thread owns one 32-column block of every row it
+// sees, so its dgamma partial sums stay in registers across rows.  At the end
+// every row group writes its partial row to the workspace; a second kernel adds
+// the partial rows in a fixed order (deterministic, no atomics).
+#pragma once
+
+#include "row_fwd.cuh"
+
+namespace mxn {
+
+struct BwdArgs {
+  const uint16_t* x;      // bf16 [T, D]
+  const uint16_t* dy;     // bf16 [T, D]
+  const uint16_t* gamma;  // bf16 [D] or null
+  const float* G;         // fp32 [T]
+  uint16_t* dx;           // bf16 [T, D]
+  float* partial;         // fp32 [gridDim.x * rps, D] or null (no dgamma)
+  unsigned* status;
+};
+
+__device__ __forceinline__ void produce_rows2(const uint16_t* x, const uint16_t* dy,
+                                              const RowCfg& C, uint8_t* stage0, uint64_t* full,
+                                              uint64_t* empty, unsigned* status) {
+  const uint64_t pol = policy_evict_first();
+  int64_t it = 0;
+  for (int64_t rb = blockIdx.x; rb < C.n_row_blocks; rb += gridDim.x, ++it) {
+    const int s = (int)(it % C.stages);
+    const uint32_t ph = (uint32_t)((it / C.stages) & 1);
+    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, status)) break;
+    const int64_t r0 = rb * C.rps;
+    const int nrows = (int)(C.T - r0 < (int64_t)C.rps ? C.T - r0 : (int64_t)C.rps);
+    mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)nrows * C.row_bytes);
+    uint8_t* dst = stage0 + (size_t)s * C.stage_bytes;
+    for (int r = 0; r < nrows; ++r) {
+      bulk_copy_g2s(dst + (size_t)r * C.row_bytes, x + (r0 + r) * C.ld_x, C.row_bytes, &full[s], pol);
+      bulk_copy_g2s(dst + (size_t)(C.rps + r) * C.row_bytes, dy + (r0 + r) * C.ld_x, C.row_bytes,
+                    &full[s], pol);
+    }
+  }
+  for (int64_t j = (it > C.stages ? it - C.stages : (int64_t)0); j < it; ++j)
+    mbar_wait_bounded(&full[j % C.stages], (uint32_t)((j / C.stages) & 1), status);
+}
+
+// Row sums of two quantities at once.
+__device__ __forceinline__ float2 row_sum2(float2 v, const RowCfg& C, float2* red, int grp, int tg,
+                                           int lane, int par) {
+  const int W = C.tpr < 32 ? C.tpr : 32;
+  v.x = seg_sum(v.x, W);
+  v.y = seg_sum(v.y, W);
+  if (C.tpr > 32) {
+    const int nw = C.tpr >> 5;
+    float2* slot = red + (par * C.rps + grp) * kRedSlots;
+    if (lane == 0) slot[tg >> 5] = v;
+    named_barrier_sync(1 + grp, C.tpr);
+    v = make_float2(0.0f, 0.0f);
+    for (int w = 0; w < nw; ++w) {
+      v.x += slot[w].x;
+      v.y += slot[w].y;
+    }
+  }
+  return v;
+}
+
+template <int NCT>
+__global__ void __launch_bounds__(CtaShape<NCT>::threads, NCT <= 128 ? 3 : 1)
+    row_bwd_kernel(const BwdArgs A, const RowCfg C) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* stage0 = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)C.stages * C.stage_bytes);
+  uint64_t* empty = full + C.stages;
+  float2* red = reinterpret_cast<float2*>(empty + C.stages);
+
+  const int tid = threadIdx.x;
+  constexpr int ncons = NCT;
+  if (tid == 0) {
+    for (int s = 0; s < C.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C.n_cwarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid >= ncons) {
+    if (tid == ncons) produce_rows2(A.x, A.dy, C, stage0, full, empty, A.status);
+    return;
+  }
+
+  const int lane = tid & 31;
+  const int grp = tid >> C.log2_tpr;
+  const int tg = tid & (C.tpr - 1);
+  const int k = tg;                       // one 32-column block per thread
+  const bool mine = k < C.K;
+  const int rot = (k >> 1) & 3;
+
+  uint32_t gw[16];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint4 v = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    if (A.gamma != nullptr && mine) v = ldg128_nc(A.gamma + (size_t)k * kBlock + ((j + rot) & 3) * 8);
+    gw[4 * j] = v.x; gw[4 * j + 1] = v.y; gw[4 * j + 2] = v.z; gw[4 * j + 3] = v.w;
+  }
+  float acc[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+
+  // x and dy stay in the stage: pass 1 reads them for the two row sums, pass 2
+  // reads them again for dx and the dgamma partials, and only then is the
+  // stage released.  That keeps the registers for the 32 dgamma accumulators.
+  bool ok = true;
+  int par = 0;
+  int64_t it = 0;
+  for (int64_t rb = blockIdx.x; rb < C.n_row_blocks; rb += gridDim.x, ++it, par ^= 1) {
+    const int s = (int)(it % C.stages);
+    const uint32_t ph = (uint32_t)((it / C.stages) & 1);
+    if (ok) ok = mbar_wait_bounded(&full[s], ph, A.status);
+    const int64_t row = rb * C.rps + grp;
+    const bool valid = row < C.T;
+    const bool have = valid && mine;
+    const uint8_t* sbase = stage0 + (size_t)s * C.stage_bytes;
+    const uint32_t sx = smem_u32(sbase + (size_t)grp * C.row_bytes) + (uint32_t)k * 64u;
+    const uint32_t sd = smem_u32(sbase + (size_t)(C.rps + grp) * C.row_bytes) + (uint32_t)k * 64u;
+
+    float2 part = make_float2(0.0f, 0.0f);  // (x . x, x . g)
+    if (have) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t off = (uint32_t)(((j + rot) & 3) * 16);
+        const uint4 a = lds128(sx + off), d = lds128(sd + off);
+        const uint32_t xa[4] = {a.x, a.y, a.z, a.w}, da[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t g2 = gw[4 * j + i];
+          const float x0 = bf16lo(xa[i]), x1 = bf16hi(xa[i]);
+          part.x = fmaf(x0, x0, part.x);
+          part.x = fmaf(x1, x1, part.x);
+          part.y = fmaf(x0, __fmul_rn(bf16lo(g2), bf16lo(da[i])), part.y);
+          part.y = fmaf(x1, __fmul_rn(bf16hi(g2), bf16hi(da[i])), part.y);
+        }
+      }
+    }
+    const float2 tot = row_sum2(part, C, red, grp, tg, lane, par);
+    if (have) {
+      const float G = __ldg(A.G + row);
+      const bool live = (G != 0.0f) && (tot.x != 0.0f);
+      const float invG = live ? __frcp_rn(G) : 0.0f;
+      const float coef = live ? tot.y / tot.x : 0.0f;
+      uint16_t* dxrow = A.dx + row * (int64_t)C.D + (int64_t)k * kBlock;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t off = (uint32_t)(((j + rot) & 3) * 16);
+        const uint4 a = lds128(sx + off), d = lds128(sd + off);
+        const uint32_t xa[4] = {a.x, a.y, a.z, a.w}, da[4] = {d.x, d.y, d.z, d.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int w = 4 * j + i;
+          const float x0 = bf16lo(xa[i]), x1 = bf16hi(xa[i]);
+          const float d0 = bf16lo(da[i]), d1 = bf16hi(da[i]);
+          const float g0 = __fmul_rn(bf16lo(gw[w]), d0), g1 = __fmul_rn(bf16hi(gw[w]), d1);
+          const float r0 = __fmul_rn(fmaf(-x0, coef, g0), invG);
+          const float r1 = __fmul_rn(fmaf(-x1, coef, g1), invG);
+          const __nv_bfloat162 h = __floats2bfloat162_rn(r0, r1);
+          o[i] = *reinterpret_cast<const uint32_t*>(&h);
+          acc[2 * w] = fmaf(__fmul_rn(d0, x0), invG, acc[2 * w]);
+          acc[2 * w + 1] = fmaf(__fmul_rn(d1, x1), invG, acc[2 * w + 1]);
+        }
+        stg128_stream(dxrow + ((j + rot) & 3) * 8, make_uint4(o[0], o[1], o[2], o[3]));
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+
+  if (A.partial != nullptr && mine) {
+    float* prow = A.partial + ((int64_t)blockIdx.x * C.rps + grp) * C.D + (int64_t)k * kBlock;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float* p = prow + ((j + rot) & 3) * 8;
+      reinterpret_cast<float4*>(p)[0] = make_float4(acc[8 * j], acc[8 * j + 1], acc[8 * j + 2], acc[8 * j + 3]);
+      reinterpret_cast<float4*>(p)[1] = make_float4(acc[8 * j + 4], acc[8 * j + 5], acc[8 * j + 6], acc[8 * j + 7]);
+    }
+  }
+}
+
+// dgamma[j] = sum over the n_part partial rows, in a fixed order: thread
+// (tx, ty) of a 32 x 32 CTA adds rows ty, ty + 32, ... of column j = 32 *
+// blockIdx.x + tx; the 32 lane sums are then added in ty order.
+__global__ void __launch_bounds__(1024) dgamma_reduce_kernel(const float* partial, int64_t n_part,
+                                                             int D, uint16_t* dgamma) {
+  __shared__ float sh[32][33];
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int j = blockIdx.x * 32 + tx;
+  float s = 0.0f;
+  if (j < D)
+    for (int64_t r = ty; r < n_part; r += 32) s += partial[r * D + j];
+  sh[ty][tx] = s;
+  __syncthreads();
+  if (ty == 0 && j < D) {
+    float t = 0.0f;
+    for (int i = 0; i < 32; ++i) t += sh[i][tx];
+    const __nv_bfloat16 h = __float2bfloat16_rn(t);
+    dgamma[j] = *reinterpret_cast<const uint16_t*>(&h);
+  }
+}
+
+}  // namespace mxn

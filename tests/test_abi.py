@@ -1,0 +1,130 @@
+"""The C-ABI library loads, exports every symbol include/mxnorm.h declares, and
+rejects bad arguments with the documented status before touching the GPU.
+
+No test here launches a kernel: invalid calls return during validation, and
+the fault-injection hook fails a call on the host before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from normalisation_row_bf16_b200 import build as nbuild
+from normalisation_row_bf16_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    nbuild.build()
+    return ops.lib()
+
+
+def _declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, re.M):
+            if m.group(1) not in ("defined",):
+                names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = _declared_functions()
+    assert "mxnorm_fwd" in names and "mxnorm_bwd" in names and len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+        assert n in ops.SIGNATURES, f"{n} has no binding"
+
+
+def test_scales_bytes(L):
+    assert ops.scales_bytes(8192, 4096, ops.SCALES_ROWMAJOR) == 8192 * 128
+    assert ops.scales_bytes(100, 4128, ops.SCALES_MMA) == 128 * 132
+    assert ops.scales_bytes(0, 64, ops.SCALES_ROWMAJOR) == 0
+    assert ops.scales_bytes(4, 33, ops.SCALES_ROWMAJOR) == 0
+    assert ops.scales_bytes(4, 64, 7) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)          # aligned, never dereferenced on these paths
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def _fwd(L, x=FAKE, q=FAKE, s=FAKE, T=4, D=64, ld=64, p=2.0, rnd=0, layout=0, gamma=None, G=None):
+    return L.mxnorm_fwd(x, gamma, q, s, G, T, D, ld, p, rnd, 0, layout, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=33), ops.MXN_ERR_ARG),
+    (dict(D=0), ops.MXN_ERR_ARG),
+    (dict(T=-1), ops.MXN_ERR_ARG),
+    (dict(ld=60), ops.MXN_ERR_ARG),
+    (dict(ld=68), ops.MXN_ERR_ARG),
+    (dict(x=None), ops.MXN_ERR_ARG),
+    (dict(q=None), ops.MXN_ERR_ARG),
+    (dict(s=None), ops.MXN_ERR_ARG),
+    (dict(x=MISALIGNED), ops.MXN_ERR_ARG),
+    (dict(gamma=MISALIGNED), ops.MXN_ERR_ARG),
+    (dict(p=0.0), ops.MXN_ERR_ARG),
+    (dict(p=-1.0), ops.MXN_ERR_ARG),
+    (dict(p=float("nan")), ops.MXN_ERR_ARG),
+    (dict(rnd=2), ops.MXN_ERR_ARG),
+    (dict(layout=2), ops.MXN_ERR_ARG),
+    (dict(D=32768 + 32, ld=32768 + 32), ops.MXN_ERR_UNSUPPORTED),
+])
+def test_fwd_argument_errors(L, kw, code):
+    assert _fwd(L, **kw) == code
+    assert L.mxnorm_last_error().decode() != ""
+
+
+def test_empty_input_is_a_noop(L):
+    assert _fwd(L, T=0) == ops.MXN_OK
+    assert L.mxfp8_cast(FAKE, FAKE, FAKE, 0, 64, 64, 0, 0, 0, None) == ops.MXN_OK
+    assert L.rmsnorm_bf16(FAKE, None, FAKE, 0, 64, 64, 1e-5, None) == ops.MXN_OK
+    assert L.mxnorm_bwd(FAKE, FAKE, None, FAKE, FAKE, None, 0, 64, None, 0, None) == ops.MXN_OK
+
+
+def test_other_entry_points_validate(L):
+    assert L.mxfp8_cast(FAKE, FAKE, FAKE, 4, 48, 48, 0, 0, 0, None) == ops.MXN_ERR_ARG
+    assert L.rmsnorm_bf16(FAKE, None, None, 4, 64, 64, 1e-5, None) == ops.MXN_ERR_ARG
+    assert L.rmsnorm_bf16(FAKE, None, FAKE, 4, 64, 64, -1.0, None) == ops.MXN_ERR_ARG
+    assert L.rmsnorm_then_mxcast(FAKE, None, 1e-5, FAKE, FAKE, FAKE, 4, 64, 64, 5, None) == ops.MXN_ERR_ARG
+    # dgamma without gamma, and a row length beyond the backward's limit
+    assert L.mxnorm_bwd(FAKE, FAKE, None, FAKE, FAKE, FAKE, 4, 64, FAKE, 1 << 20, None) == ops.MXN_ERR_ARG
+    assert L.mxnorm_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, 4, 32768, None, 0, None) == ops.MXN_ERR_UNSUPPORTED
+    assert L.mxnorm_bwd(FAKE, FAKE, None, MISALIGNED, FAKE, None, 4, 64, None, 0, None) == ops.MXN_ERR_ARG
+    assert L.mxnorm_bwd_workspace_size(4, 33) == 0
+
+
+def test_tuning_validation(L):
+    assert L.mxnorm_set_tuning(96, 0, 0) == ops.MXN_ERR_ARG
+    assert L.mxnorm_set_tuning(0, 1, 0) == ops.MXN_ERR_ARG
+    assert L.mxnorm_set_tuning(0, 0, 9) == ops.MXN_ERR_ARG
+    assert L.mxnorm_set_tuning(256, 4, 2) == ops.MXN_OK
+    assert L.mxnorm_set_tuning(0, 0, 0) == ops.MXN_OK
+
+
+def test_host_fault_injection(L):
+    """The hook makes the next calls fail on the host with MXN_ERR_CUDA, after
+    argument checks and before any CUDA call; then calls behave again."""
+    L.mxnorm_debug_fail_next(2)
+    assert _fwd(L) == ops.MXN_ERR_CUDA
+    assert "injected" in L.mxnorm_last_error().decode()
+    assert L.mxfp8_cast(FAKE, FAKE, FAKE, 4, 64, 64, 0, 0, 0, None) == ops.MXN_ERR_CUDA
+    # invalid arguments are still reported as such while injection is armed
+    L.mxnorm_debug_fail_next(1)
+    assert _fwd(L, D=33) == ops.MXN_ERR_ARG
+    L.mxnorm_debug_fail_next(0)
+    assert _fwd(L, T=0) == ops.MXN_OK
+
+
+def test_python_binding_refuses_cpu_tensors(L):
+    import torch
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ops.mxnorm_fwd(x)
