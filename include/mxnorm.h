@@ -172,10 +172,13 @@ const char* mxnorm_last_error(void);
 int mxnorm_device_status(void* stream);
 
 /*
- * Launch tuning for the row kernels (all four ops): consumer threads per CTA
- * (128, 256 or 512), pipeline stages (2..16) and CTAs per SM (1..8); 0 keeps
- * the library's choice.  Process-wide; not thread-safe against concurrent
- * launches.  Returns MXN_ERR_ARG for out-of-range values.
+ * Launch tuning for the row kernels: threads per CTA (a multiple of 32 up to
+ * 512; the forward kernels split them into row groups, the backward uses them
+ * as consumer threads and accepts 128, 256 or 512), shared-memory stages per
+ * pipeline (1..16) and CTAs per SM (1..8); 0 keeps the library's choice.
+ * Process-wide; not thread-safe against concurrent launches.  Returns
+ * MXN_ERR_ARG for out-of-range values; a shape that does not fit an SM makes
+ * the next launch return MXN_ERR_UNSUPPORTED.
  */
 int mxnorm_set_tuning(int consumer_threads, int stages, int ctas_per_sm);
 

@@ -193,8 +193,13 @@ int launch(const Plan& P, void* args, cudaStream_t stream) {
   return MXN_OK;
 }
 
+// Pointer checks are skipped for T = 0 (an empty tensor may have no storage);
+// shape checks always run.
+thread_local bool t_empty = false;
+
 int check_common(const void* x, int64_t T, int64_t D, int64_t ld_x) {
-  if (!x) return fail(MXN_ERR_ARG, "x is NULL");
+  t_empty = (T == 0);
+  if (!x && !t_empty) return fail(MXN_ERR_ARG, "x is NULL");
   if (T < 0) return fail(MXN_ERR_ARG, "T = %lld < 0", (long long)T);
   if (D <= 0 || D % kBlock != 0) return fail(MXN_ERR_ARG, "D = %lld is not a positive multiple of 32", (long long)D);
   if (D > MXN_MAX_D) return fail(MXN_ERR_UNSUPPORTED, "D = %lld > %d", (long long)D, MXN_MAX_D);
@@ -205,6 +210,7 @@ int check_common(const void* x, int64_t T, int64_t D, int64_t ld_x) {
 }
 
 int check_out(const void* p, const char* name) {
+  if (!p && t_empty) return MXN_OK;
   if (!p) return fail(MXN_ERR_ARG, "%s is NULL", name);
   if (!aligned16(p)) return fail(MXN_ERR_ARG, "%s is not 16-byte aligned", name);
   return MXN_OK;
@@ -215,15 +221,116 @@ int check_opt(const void* p, const char* name) {
   return MXN_OK;
 }
 
+// The instantiation for (blocks per thread, threads per row): 32 threads per
+// row for up to 4 blocks each (D <= 4096), 64..256 threads with 4 blocks each
+// beyond, a runtime segment width below 32 blocks per row.
 template <int MODE, bool SR>
-const void* fwd_kernel(int bpt, int nct) {
-  if (bpt == 2) return (const void*)row_fwd_kernel<MODE, 2, 512, SR>;
-  switch (nct) {
-    case 128: return (const void*)row_fwd_kernel<MODE, 1, 128, SR>;
-    case 256: return (const void*)row_fwd_kernel<MODE, 1, 256, SR>;
-    case 512: return (const void*)row_fwd_kernel<MODE, 1, 512, SR>;
+const void* fwd_kernel(int bpt, int tpr) {
+  if (tpr < 32) return bpt == 1 ? (const void*)row_fwd_kernel<MODE, 1, 0, SR> : nullptr;
+  if (tpr == 32) {
+    switch (bpt) {
+      case 1: return (const void*)row_fwd_kernel<MODE, 1, 32, SR>;
+      case 2: return (const void*)row_fwd_kernel<MODE, 2, 32, SR>;
+      case 4: return (const void*)row_fwd_kernel<MODE, 4, 32, SR>;
+      default: return nullptr;
+    }
+  }
+  if (bpt != 4) return nullptr;
+  switch (tpr) {
+    case 64: return (const void*)row_fwd_kernel<MODE, 4, 64, SR>;
+    case 128: return (const void*)row_fwd_kernel<MODE, 4, 128, SR>;
+    case 256: return (const void*)row_fwd_kernel<MODE, 4, 256, SR>;
     default: return nullptr;
   }
+}
+
+// Launch plan for the forward row kernels (row_fwd.cuh).
+struct FwdPlan {
+  FwdCfg C;
+  const void* kernel = nullptr;
+  int threads = 0;
+  size_t smem = 0;
+  int grid = 0;
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int plan_fwd(int mode, bool sr, bool gamma_smem, int64_t T, int D, int64_t ld_x, int sms, FwdPlan* P) {
+  FwdCfg& C = P->C;
+  C = FwdCfg{};
+  C.T = T;
+  C.ld_x = ld_x;
+  C.D = D;
+  C.K = D / kBlock;
+  // Blocks per thread and threads per row: rows of up to 128 blocks take one
+  // warp (1, 2 or 4 blocks per thread), longer rows 4 blocks per thread over
+  // 64..256 threads, rows under 32 blocks a power-of-two segment of a warp.
+  int bpt;
+  if (C.K <= 32) { bpt = 1; C.tpr = next_pow2(C.K); }
+  else if (C.K <= 64) { bpt = 2; C.tpr = 32; }
+  else if (C.K <= 128) { bpt = 4; C.tpr = 32; }
+  else { bpt = 4; C.tpr = next_pow2((C.K + 3) / 4); }
+  C.log2_tpr = ilog2(C.tpr);
+  C.gthreads = C.tpr < 32 ? 32 : C.tpr;
+  C.rps = C.gthreads / C.tpr;
+  C.row_bytes = 2u * (uint32_t)D;
+  C.stage_bytes = (uint32_t)C.rps * C.row_bytes;
+  // Default: as many single-row groups as the CTA holds (up to 24 warps), and
+  // extra stages only while 176 KB of shared memory still covers them all.
+  if (g_tuning.stages) {
+    C.stages = g_tuning.stages;
+  } else {
+    const int gmax = fwd_max_threads(bpt) / (C.tpr < 32 ? 32 : C.tpr);
+    int st = (int)((176u * 1024u) / ((size_t)gmax * C.rps * 2u * (uint32_t)D));
+    C.stages = st < 1 ? 1 : (st > 3 ? 3 : st);
+  }
+  C.gamma_f32 = D <= 8192 ? 1 : 0;
+  C.gamma_bytes = gamma_smem ? (uint32_t)align_up((C.gamma_f32 ? 4u : 2u) * (uint32_t)D, 128) : 0u;
+  const size_t per_group = (size_t)C.stages * C.stage_bytes;
+  // Shared memory per group: its ring, its 2 * stages barriers and its two
+  // reduction slot arrays; plus gamma and 16 bytes of alignment once.
+  const size_t per_group_all = per_group + (size_t)2 * C.stages * sizeof(uint64_t) +
+                               (size_t)2 * kRedSlots * sizeof(float2);
+  int ng;
+  if (g_tuning.consumer_threads) {
+    ng = g_tuning.consumer_threads / C.gthreads;
+  } else {
+    ng = fwd_max_threads(bpt) / C.gthreads;
+  }
+  int ng_max = fwd_max_threads(bpt) / C.gthreads;
+  const size_t fixed = C.gamma_bytes + 16;
+  const size_t smem_cap = 227u * 1024u;
+  if (fixed + per_group_all > smem_cap)
+    return fail(MXN_ERR_UNSUPPORTED, "row of %d elements does not fit in shared memory", D);
+  const int ng_fit = (int)((smem_cap - fixed) / per_group_all);
+  if (ng_fit < ng_max) ng_max = ng_fit;
+  ng = ng < 1 ? 1 : (ng > ng_max ? ng_max : ng);
+  if (C.tpr > 32 && ng > 15) ng = 15;  // named barriers 1..15
+  C.ng = ng;
+  C.n_row_blocks = (T + C.rps - 1) / C.rps;
+  C.ring_off = C.gamma_bytes;
+  C.bar_off = (uint32_t)align_up(C.ring_off + (size_t)ng * per_group, 16);
+  C.red_off = C.bar_off + (uint32_t)(ng * 2 * C.stages * sizeof(uint64_t));
+  P->smem = C.red_off + (size_t)ng * 2 * kRedSlots * sizeof(float2);
+  P->threads = ng * C.gthreads;
+  P->kernel = sr ? (mode == kModeMXNorm ? fwd_kernel<kModeMXNorm, true>(bpt, C.tpr)
+                                        : fwd_kernel<kModeCast, true>(bpt, C.tpr))
+                 : (mode == kModeMXNorm ? fwd_kernel<kModeMXNorm, false>(bpt, C.tpr)
+                    : mode == kModeCast ? fwd_kernel<kModeCast, false>(bpt, C.tpr)
+                                        : fwd_kernel<kModeRMSNorm, false>(bpt, C.tpr));
+  if (!P->kernel) return fail(MXN_ERR_UNSUPPORTED, "no kernel for D = %d", D);
+  int occ = 0;
+  int rc = occupancy(P->kernel, P->threads, P->smem, &occ);
+  if (rc) return rc;
+  if (occ < 1) return fail(MXN_ERR_UNSUPPORTED, "row kernel does not fit on an SM (D = %d)", D);
+  if (g_tuning.ctas_per_sm && g_tuning.ctas_per_sm < occ) occ = g_tuning.ctas_per_sm;
+  // One CTA per resident slot (fewer when there are fewer row blocks than groups).
+  const int64_t max_ctas = (int64_t)sms * occ;
+  const int64_t need_ctas = (C.n_row_blocks + ng - 1) / ng;
+  const int64_t ctas = need_ctas < max_ctas ? need_ctas : max_ctas;
+  C.ngt = ctas * ng;
+  P->grid = (int)ctas;
+  return MXN_OK;
 }
 
 const void* bwd_kernel(int bpt, int nct) {
@@ -236,19 +343,21 @@ const void* bwd_kernel(int bpt, int nct) {
   }
 }
 
-template <int MODE>
-int launch_fwd(const FwdArgs& A, int64_t T, int D, int64_t ld_x, cudaStream_t stream) {
+int launch_fwd(int mode, bool sr, const FwdArgs& A, int64_t T, int D, int64_t ld_x,
+               cudaStream_t stream) {
   DeviceInfo dev;
   int rc = device_info(&dev);
   if (rc) return rc;
-  Plan P;
-  KernelPicker pick = A.sr ? fwd_kernel<MODE, true> : fwd_kernel<MODE, false>;
-  if (MODE == kModeRMSNorm) pick = fwd_kernel<MODE, false>;
-  rc = plan_rows(T, D, ld_x, 1, pick, dev.sms, &P);
+  FwdPlan P;
+  rc = plan_fwd(mode, sr, A.gamma != nullptr && mode != kModeCast, T, D, ld_x, dev.sms, &P);
   if (rc) return rc;
   FwdArgs a = A;
   a.status = dev.status;
-  return launch(P, &a, stream);
+  a.inv_K = 1.0f / (float)(D / kBlock);
+  void* argv[] = {&a, &P.C};
+  cudaError_t e = cudaLaunchKernel(P.kernel, dim3(P.grid), dim3(P.threads), argv, P.smem, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "row_fwd_kernel launch");
+  return MXN_OK;
 }
 
 int pmode_of(float p) {
@@ -301,14 +410,12 @@ static int fwd_like(int mode, const void* x, const void* gamma, void* q, void* s
   A.p = p;
   A.inv_p = std::isinf(p) ? 0.0f : 1.0f / p;
   A.pmode = pmode_of(p);
-  A.sr = rounding == MXN_ROUND_SR;
   A.seed_lo = (uint32_t)seed;
   A.seed_hi = (uint32_t)(seed >> 32);
   A.scale_mma = scale_layout == MXN_SCALES_MMA;
   A.kp4 = (int)(((D / kBlock) + 3) / 4 * 4);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return mode == kModeMXNorm ? launch_fwd<kModeMXNorm>(A, T, (int)D, ld_x, s)
-                             : launch_fwd<kModeCast>(A, T, (int)D, ld_x, s);
+  return launch_fwd(mode, rounding == MXN_ROUND_SR, A, T, (int)D, ld_x, s);
 }
 
 int mxnorm_fwd(const void* x, const void* gamma, void* q, void* scales, float* G_out, int64_t T,
@@ -339,7 +446,7 @@ int rmsnorm_bf16(const void* x, const void* gamma, void* y, int64_t T, int64_t D
   A.gamma = static_cast<const uint16_t*>(gamma);
   A.y = static_cast<uint16_t*>(y);
   A.eps = eps;
-  return launch_fwd<kModeRMSNorm>(A, T, (int)D, ld_x, static_cast<cudaStream_t>(stream));
+  return launch_fwd(kModeRMSNorm, false, A, T, (int)D, ld_x, static_cast<cudaStream_t>(stream));
 }
 
 int rmsnorm_then_mxcast(const void* x, const void* gamma, float eps, void* y_tmp, void* q,
@@ -435,10 +542,9 @@ int mxnorm_device_status(void* stream) {
 
 int mxnorm_set_tuning(int consumer_threads, int stages, int ctas_per_sm) {
   t_err.clear();
-  if (consumer_threads != 0 && consumer_threads != 128 && consumer_threads != 256 &&
-      consumer_threads != 512)
+  if (consumer_threads != 0 && (consumer_threads < 32 || consumer_threads > 512 || consumer_threads % 32))
     return fail(MXN_ERR_ARG, "consumer_threads = %d", consumer_threads);
-  if (stages != 0 && (stages < 2 || stages > 16)) return fail(MXN_ERR_ARG, "stages = %d", stages);
+  if (stages != 0 && (stages < 1 || stages > 16)) return fail(MXN_ERR_ARG, "stages = %d", stages);
   if (ctas_per_sm < 0 || ctas_per_sm > 8) return fail(MXN_ERR_ARG, "ctas_per_sm = %d", ctas_per_sm);
   g_tuning.consumer_threads = consumer_threads;
   g_tuning.stages = stages;

@@ -62,14 +62,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the warp sleeps until the phase
+// completes or about `hint_ns` pass, instead of spinning on issue slots that
+// the computing warps need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase of `bar` with the given parity has completed, for at
 // most kWaitLimitNs.  Returns false (and records the timeout in *status) if
-// the wait gave up.
+// the wait gave up.  Sleeping waits: the clock is read once per ~20 us wake-up.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   unsigned* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       atomicOr(status, kStatusWaitTimeout);
       return false;
@@ -152,6 +167,56 @@ __device__ __forceinline__ float bf16bits_to_float(uint32_t b16) { return __uint
 // 2^n for an integer n in [-126, 127], built from its exponent field.
 __device__ __forceinline__ float exp2_int(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): each call is one instruction
+// doing two correctly rounded fp32 multiplies.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<const float2*>(&d);
+}
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
+        "l"(*reinterpret_cast<const uint64_t*>(&c)));
+  return *reinterpret_cast<const float2*>(&d);
+}
+
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) { return make_float2(bf16lo(w), bf16hi(w)); }
+
+// max(a, |b|, |c|), propagating NaN.
+__device__ __forceinline__ float max3_abs_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+  return d;
+}
+
+// Packed bf16 pair whose halves are the larger magnitudes of a's and b's
+// halves (signs are junk; NaN propagates).  Folding 16 words with it gives the
+// block absmax in 15 instructions.
+__device__ __forceinline__ uint32_t bf16x2_maxabs(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Magnitude bits (bf16, low 16 bits) of the absmax of 16 packed words.
+__device__ __forceinline__ uint32_t block_absmax16(const uint32_t* w) {
+  uint32_t a0 = bf16x2_maxabs(w[0], w[1]), a1 = bf16x2_maxabs(w[2], w[3]);
+  uint32_t a2 = bf16x2_maxabs(w[4], w[5]), a3 = bf16x2_maxabs(w[6], w[7]);
+  uint32_t a4 = bf16x2_maxabs(w[8], w[9]), a5 = bf16x2_maxabs(w[10], w[11]);
+  uint32_t a6 = bf16x2_maxabs(w[12], w[13]), a7 = bf16x2_maxabs(w[14], w[15]);
+  a0 = bf16x2_maxabs(a0, a1); a2 = bf16x2_maxabs(a2, a3);
+  a4 = bf16x2_maxabs(a4, a5); a6 = bf16x2_maxabs(a6, a7);
+  a0 = bf16x2_maxabs(a0, a2); a4 = bf16x2_maxabs(a4, a6);
+  a0 = bf16x2_maxabs(a0, a4);
+  return max(a0 & 0x7FFFu, (a0 >> 16) & 0x7FFFu);
+}
+
 // ------------------------------------------------------------------ E8M0 scale
 
 // Scale exponent of a block whose absmax has fp32 bits `abits` (non-negative):
@@ -174,6 +239,19 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2_rn(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return (uint32_t)r;
+}
+
+// Four fp32 -> four E4M3 codes (nearest even, saturating finite), packed with
+// the code of `a` in bits 0..7 through `d` in bits 24..31.
+__device__ __forceinline__ uint32_t cvt_e4m3x4_rn(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 l, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;\n\t"
+      "mov.b32 %0, {l, h};\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
 }
 
 // ---------------------------------------------------------- Philox4x32-10

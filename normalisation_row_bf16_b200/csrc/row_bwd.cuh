@@ -20,6 +20,30 @@
 
 namespace mxn {
 
+constexpr int kMaxConsumerThreads = 512;
+
+// Launch shape of the backward: one consumer thread per 32-column block, rows
+// grouped rps per stage, one producer warp per CTA.
+struct RowCfg {
+  int64_t T;             // rows
+  int64_t ld_x;          // row stride of the input, elements
+  int64_t n_row_blocks;  // ceil(T / rps)
+  int D, K;              // row length, blocks per row
+  int tpr, log2_tpr;     // consumer threads per row (power of two)
+  int rps;               // rows per stage
+  int stages;            // pipeline depth
+  int n_cwarps;          // consumer warps
+  uint32_t row_bytes;    // 2 * D
+  uint32_t stage_bytes;  // rps * row_bytes * 2 (x and dy)
+};
+
+// Resident CTAs per SM the register budget is sized for, by consumer threads
+// per CTA (each CTA adds one producer warp).
+template <int NCT>
+struct CtaShape {
+  static constexpr int threads = NCT + 32;
+};
+
 struct BwdArgs {
   const uint16_t* x;      // bf16 [T, D]
   const uint16_t* dy;     // bf16 [T, D]

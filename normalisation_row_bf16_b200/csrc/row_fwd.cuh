@@ -1,28 +1,35 @@
-// row_fwd.cuh -- the single-input row kernels: MXNorm forward, MXCast and the
+// row_fwd.cuh -- the forward row kernels: MXNorm forward, MXCast and the
 // RMSNorm pass of the two-pass comparator.
 //
 // MXNorm (gist.science, "MXNorm: Reusing MXFP block scales for efficient
 // tensor normalisation", technical summary section 2.1) reads each row once:
 // block absmax m_k -> generalised p-mean G -> y = x / G (* gamma) -> E8M0
-// scale per block -> E4M3 codes.  The pages' own kernel ran through
-// torch.compile on GB200 (section 3.2); this one is written for B200:
+// scale per block -> E4M3 codes.  The pages ran theirs through torch.compile
+// on GB200 (section 3.2); this one is laid out for B200:
 //
-//  * persistent CTAs (grid = SMs x resident CTAs), each owning a strided set
-//    of "row blocks" (rps consecutive rows);
-//  * one producer thread streams whole rows into a ring of shared-memory
-//    stages with 1-D bulk copies on the TMA engine (cp.async.bulk, no
-//    multicast, L2 evict-first), so the bytes in flight do not depend on
-//    register-file occupancy;
-//  * consumer threads own one 32-element MX block each (bpt blocks when the
-//    row has more than 512 blocks), so the block absmax, scale and cast are
-//    thread-local; the row statistic is a K-input reduction (warp shuffles,
-//    then one named barrier across the row's warps): K = D/32 inputs, the
-//    32x smaller reduction the lay summary (section 3) points at;
-//  * a thread reads its 64 bytes as four 16-byte chunks in a rotated order
-//    (chunk (j + k/2) mod 4 at step j) so that the eight threads of a
-//    shared-memory phase hit eight distinct 16-byte bank groups;
-//  * each stage is released (mbarrier arrive) as soon as its data sit in
-//    registers, before the arithmetic, so the next copy overlaps it.
+//  * A "row group" of tpr threads owns one row at a time (tpr = 32 up to
+//    D = 4096, i.e. one warp per row; more warps per row beyond that; several
+//    rows per warp below D = 1024).  Each thread owns BPT of the row's 32-element
+//    MX blocks (k = tg + b * tpr), so the block absmax, scale and cast are
+//    thread-local and the row statistic reduces K = D/32 numbers -- with warp
+//    shuffles only when the row fits one warp (the lay summary's "32x less
+//    reduction work", section 3).
+//  * Each row group owns a ring of `stages` shared-memory row buffers filled by
+//    1-D bulk copies (cp.async.bulk on the TMA engine, L2 evict-first, no
+//    multicast) that its first thread issues, completing on the group's own
+//    mbarriers: no group ever waits for another, and the bytes in flight do not
+//    depend on register occupancy.
+//  * A thread copies its blocks from the stage into registers and hands the
+//    stage straight back; the refill (row block rb + stages * ngt) is issued
+//    before the row's arithmetic, so each group keeps `stages` rows of compute
+//    as look-ahead whatever the occupancy.  A thread reads its 64-byte block
+//    as four 16-byte chunks in the order (j + k/2) mod 4, which puts the eight
+//    threads of a shared-memory phase on eight distinct bank groups.
+//  * gamma is converted once per CTA into shared memory in "slot order": the
+//    16 bytes that match x chunk slot j of block k sit at (j * K + k) * 16, so
+//    consecutive threads read consecutive 16-byte words.
+//  * fp32 products run as packed f32x2 multiplies (two IEEE-rounded products
+//    per instruction), the per-block maxima as 3-input max and bf16x2 max.
 #pragma once
 
 #include "device_common.cuh"
@@ -32,28 +39,28 @@ namespace mxn {
 enum RowMode { kModeMXNorm = 0, kModeCast = 1, kModeRMSNorm = 2 };
 enum PMode { kP1 = 1, kP2 = 2, kP4 = 4, kPInf = 0, kPGeneral = 3 };
 
-constexpr int kMaxConsumerThreads = 512;
-constexpr int kRedSlots = 16;  // warps per row, at most
+// Threads per CTA the register budget is sized for: a thread holding 4 blocks
+// of its row needs ~120 registers (512 threads), 2 blocks ~96 (640), 1 block
+// fits in 80 (768).
+constexpr int fwd_max_threads(int bpt) { return bpt >= 4 ? 512 : (bpt == 2 ? 640 : 768); }
+constexpr int kRedSlots = 16;  // warps per row group, at most
 
-// Resident CTAs per SM the register budget is sized for, by consumer threads
-// per CTA (each CTA adds one producer warp).
-template <int NCT>
-struct CtaShape {
-  static constexpr int threads = NCT + 32;
-  static constexpr int min_blocks = NCT <= 128 ? 4 : (NCT <= 256 ? 2 : 1);
-};
-
-struct RowCfg {
+struct FwdCfg {
   int64_t T;             // rows
-  int64_t ld_x;          // row stride of the input, elements
+  int64_t ld_x;          // row stride of x, elements
   int64_t n_row_blocks;  // ceil(T / rps)
-  int D, K;              // row length, blocks per row
-  int tpr, log2_tpr;     // consumer threads per row (power of two)
-  int rps;               // rows per stage
-  int stages;            // pipeline depth
-  int n_cwarps;          // consumer warps
+  int64_t ngt;           // row groups in the grid
+  int D, K;              // row length, MX blocks per row
+  int tpr, log2_tpr;     // threads per row (power of two)
+  int rps;               // rows per row group and stage (> 1 only when tpr < 32)
+  int gthreads;          // threads per row group = max(tpr, 32)
+  int ng;                // row groups per CTA
+  int stages;            // ring depth per group
   uint32_t row_bytes;    // 2 * D
   uint32_t stage_bytes;  // rps * row_bytes
+  uint32_t gamma_bytes;  // shared-memory gamma (0 when unused)
+  int gamma_f32;         // gamma held as fp32 (else bf16) in shared memory
+  uint32_t ring_off, bar_off, red_off;
 };
 
 struct FwdArgs {
@@ -64,9 +71,8 @@ struct FwdArgs {
   float* G_out;           // fp32 [T] or null        (MXNorm)
   uint16_t* y;            // bf16 [T, D]             (RMSNorm)
   unsigned* status;       // device status word
-  float p, inv_p, eps;
+  float p, inv_p, eps, inv_K;
   int pmode;
-  int sr;
   uint32_t seed_lo, seed_hi;
   int scale_mma;          // scales in the tcgen05 128x4 layout
   int kp4;                // K rounded up to a multiple of 4 (MMA layout)
@@ -78,8 +84,6 @@ __device__ __forceinline__ int64_t mma_scale_offset(int64_t row, int k, int kp4)
          (k & 3);
 }
 
-// 2^n for integer n <= 0; 0 below the normal range (those terms are < 2^-126
-// of the row's largest term and do not register in an fp32 sum).
 __device__ __forceinline__ float exp2_int_or_zero(int n) { return n < -126 ? 0.0f : exp2_int(n); }
 
 __device__ __forceinline__ float pow_p(float r, int pmode, float p) {
@@ -91,8 +95,8 @@ __device__ __forceinline__ float pow_p(float r, int pmode, float p) {
   }
 }
 
-// Factor 2^(p * d) that rescales a partial sum taken relative to 2^(E + d) to
-// one taken relative to 2^E (d <= 0).
+// 2^(p * d): rescales a partial sum taken relative to 2^(E + d) to one taken
+// relative to 2^E (d <= 0).  Exact for p = 1, 2, 4.
 __device__ __forceinline__ float rescale_factor(int d, int pmode, float p) {
   switch (pmode) {
     case kP1: return exp2_int_or_zero(d);
@@ -112,8 +116,7 @@ __device__ __forceinline__ float inv_pow2(int E) {
   return E == 127 ? __uint_as_float(0x00400000u) : exp2_int(-E);
 }
 
-template <typename T>
-__device__ __forceinline__ T seg_max_u32(T v, int width) {
+__device__ __forceinline__ uint32_t seg_max(uint32_t v, int width) {
   for (int off = width >> 1; off > 0; off >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
   return v;
 }
@@ -122,299 +125,399 @@ __device__ __forceinline__ float seg_sum(float v, int width) {
   return v;
 }
 
-// The row statistic G from this thread's block maxima (bf16 magnitude bits).
-// Warp partials are taken relative to the warp maximum's power of two, so no
-// term overflows or underflows; partials of different warps are combined by
-// exact power-of-two factors (integer p) after one named barrier.
-template <int BPT>
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+  uint32_t r;
+  asm("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+  return r;
+}
+
+// G from this thread's block maxima (bf16 magnitude bits).  Partials are taken
+// relative to the warp maximum's power of two, so no term over- or underflows;
+// warps of one row combine their partials by exact power-of-two factors
+// (integer p) after one named barrier.  M is combined on its bits (NaN wins).
+// The root uses sqrt.approx (relative error <= 2^-23): G is a statistic with a
+// 1e-6 tolerance; every value derived from it uses its fp32 bits exactly.
+template <int BPT, int TPR>
 __device__ __forceinline__ float row_pmean(const uint32_t (&mb)[BPT], const FwdArgs& A,
-                                           const RowCfg& C, float2* red, int grp, int tg,
-                                           int lane, int par) {
-  uint32_t mloc = 0;
+                                           const FwdCfg& C, float2* red, int bar_id, int wig,
+                                           int lane) {
+  uint32_t mloc = mb[0];
 #pragma unroll
-  for (int b = 0; b < BPT; ++b) mloc = max(mloc, mb[b]);
-  const int W = C.tpr < 32 ? C.tpr : 32;
-  mloc = seg_max_u32(mloc, W);
+  for (int b = 1; b < BPT; ++b) mloc = max(mloc, mb[b]);
+  const int W = TPR ? 32 : C.tpr;
+  mloc = TPR ? warp_max_u32(mloc) : seg_max(mloc, W);
   const float Mw = bf16bits_to_float(mloc);
+  const int Ew = norm_exponent(Mw);
   float sw = 0.0f;
-  if (A.pmode != kPInf) {
-    const float inv = inv_pow2(norm_exponent(Mw));
+  if (A.pmode == kP2) {
+    const float inv = inv_pow2(Ew);
+#pragma unroll
+    for (int b = 0; b < BPT; ++b) {
+      const float r = bf16bits_to_float(mb[b]) * inv;
+      sw = fmaf(r, r, sw);
+    }
+    sw = seg_sum(sw, W);
+  } else if (A.pmode != kPInf) {
+    const float inv = inv_pow2(Ew);
 #pragma unroll
     for (int b = 0; b < BPT; ++b) sw += pow_p(bf16bits_to_float(mb[b]) * inv, A.pmode, A.p);
     sw = seg_sum(sw, W);
   }
   float M = Mw, S = sw;
-  int E = norm_exponent(Mw);
-  if (C.tpr > 32) {
-    const int nw = C.tpr >> 5;
-    float2* slot = red + (par * C.rps + grp) * kRedSlots;
-    if (lane == 0) slot[tg >> 5] = make_float2(Mw, sw);
-    named_barrier_sync(1 + grp, C.tpr);
+  int E = Ew;
+  if (TPR > 32) {
+    const int nw = TPR >> 5;
+    if (lane == 0) red[wig] = make_float2(Mw, sw);
+    named_barrier_sync(bar_id, TPR);
     uint32_t mb_all = 0;
-    for (int w = 0; w < nw; ++w) mb_all = max(mb_all, __float_as_uint(slot[w].x));
+#pragma unroll
+    for (int w = 0; w < nw; ++w) mb_all = max(mb_all, __float_as_uint(red[w].x));
     M = __uint_as_float(mb_all);
     E = norm_exponent(M);
     S = 0.0f;
     if (A.pmode != kPInf)
+#pragma unroll
       for (int w = 0; w < nw; ++w) {
-        const float2 v = slot[w];
+        const float2 v = red[w];
         S += v.y * rescale_factor(norm_exponent(v.x) - E, A.pmode, A.p);
       }
   }
   if (__float_as_uint(M) >= 0x7F800000u || A.pmode == kPInf) return M;  // inf / NaN / p = inf
-  const float r = S / (float)C.K;
+  const float r = S * A.inv_K;
   float root;
   switch (A.pmode) {
     case kP1: root = r; break;
-    case kP2: root = sqrtf(r); break;
-    case kP4: root = sqrtf(sqrtf(r)); break;
+    case kP2: asm("sqrt.approx.f32 %0, %1;" : "=f"(root) : "f"(r)); break;
+    case kP4: { float q; asm("sqrt.approx.f32 %0, %1;" : "=f"(q) : "f"(r));
+                asm("sqrt.approx.f32 %0, %1;" : "=f"(root) : "f"(q)); } break;
     default: root = powf(r, A.inv_p); break;
   }
   return root * exp2_int(E);
 }
 
-__device__ __forceinline__ float row_sum(float v, const RowCfg& C, float2* red, int grp, int tg,
-                                         int lane, int par) {
-  const int W = C.tpr < 32 ? C.tpr : 32;
+template <int TPR>
+__device__ __forceinline__ float row_sum(float v, const FwdCfg& C, float2* red, int bar_id,
+                                         int wig, int lane) {
+  const int W = TPR ? 32 : C.tpr;
   v = seg_sum(v, W);
-  if (C.tpr > 32) {
-    const int nw = C.tpr >> 5;
-    float2* slot = red + (par * C.rps + grp) * kRedSlots;
-    if (lane == 0) slot[tg >> 5] = make_float2(v, 0.0f);
-    named_barrier_sync(1 + grp, C.tpr);
+  if (TPR > 32) {
+    const int nw = TPR >> 5;
+    if (lane == 0) red[wig] = make_float2(v, 0.0f);
+    named_barrier_sync(bar_id, TPR);
     v = 0.0f;
-    for (int w = 0; w < nw; ++w) v += slot[w].x;
+#pragma unroll
+    for (int w = 0; w < nw; ++w) v += red[w].x;
   }
   return v;
 }
 
-// Producer: one thread streams row blocks into the stage ring.
-__device__ __forceinline__ void produce_rows(const uint16_t* x, const RowCfg& C, uint8_t* stage0,
-                                             uint64_t* full, uint64_t* empty, unsigned* status) {
-  const uint64_t pol = policy_evict_first();
-  int64_t it = 0;
-  for (int64_t rb = blockIdx.x; rb < C.n_row_blocks; rb += gridDim.x, ++it) {
-    const int s = (int)(it % C.stages);
-    const uint32_t ph = (uint32_t)((it / C.stages) & 1);
-    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, status)) break;
-    const int64_t r0 = rb * C.rps;
-    const int nrows = (int)(C.T - r0 < (int64_t)C.rps ? C.T - r0 : (int64_t)C.rps);
-    mbar_arrive_expect_tx(&full[s], (uint32_t)nrows * C.row_bytes);
-    uint8_t* dst = stage0 + (size_t)s * C.stage_bytes;
-    for (int r = 0; r < nrows; ++r)
-      bulk_copy_g2s(dst + (size_t)r * C.row_bytes, x + (r0 + r) * C.ld_x, C.row_bytes, &full[s], pol);
-  }
-  // Leave no copy in flight: wait for the last issued phase of every stage.
-  for (int64_t j = (it > C.stages ? it - C.stages : (int64_t)0); j < it; ++j)
-    mbar_wait_bounded(&full[j % C.stages], (uint32_t)((j / C.stages) & 1), status);
+// Issue the bulk copies of row block rb into `dst`, completing on `bar`.
+__device__ __forceinline__ void issue_row_block(const uint16_t* x, const FwdCfg& C, int64_t rb,
+                                                uint8_t* dst, uint64_t* bar, uint64_t pol) {
+  const int64_t r0 = rb * C.rps;
+  const int nrows = (int)(C.T - r0 < (int64_t)C.rps ? C.T - r0 : (int64_t)C.rps);
+  mbar_arrive_expect_tx(bar, (uint32_t)nrows * C.row_bytes);
+  for (int r = 0; r < nrows; ++r)
+    bulk_copy_g2s(dst + (size_t)r * C.row_bytes, x + (r0 + r) * C.ld_x, C.row_bytes, bar, pol);
 }
 
-template <int MODE, int BPT, int NCT, bool SR>
-__global__ void __launch_bounds__(CtaShape<NCT>::threads, CtaShape<NCT>::min_blocks)
-    row_fwd_kernel(const FwdArgs A, const RowCfg C) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* stage0 = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)C.stages * C.stage_bytes);
-  uint64_t* empty = full + C.stages;
-  float2* red = reinterpret_cast<float2*>(empty + C.stages);
+// The E4M3 codes of one block: 8 words, word 2j + h holding elements
+// 8c + 4h .. 8c + 4h + 3 of the chunk c that slot j holds.  Returns the
+// scale byte.  y are the block's 32 fp32 values in slot order, a their
+// absmax (>= 0 or NaN).
+template <bool SR>
+__device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a, int rot,
+                                                  uint64_t idx0, uint32_t sk0, uint32_t sk1,
+                                                  uint32_t (&qw)[8]) {
+  const int e = e8m0_exponent_bits(__float_as_uint(a) & 0x7FFFFFFFu);
+  if (e == 128) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qw[i] = 0x7F7F7F7Fu;
+    return 0xFF;
+  }
+  const float inv = exp2_int(-e);
+  const float2 inv2 = make_float2(inv, inv);
+  if constexpr (!SR) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 v0 = mul2(make_float2(y[4 * i], y[4 * i + 1]), inv2);
+      const float2 v1 = mul2(make_float2(y[4 * i + 2], y[4 * i + 3]), inv2);
+      qw[i] = cvt_e4m3x4_rn(v0.x, v0.y, v1.x, v1.y);
+    }
+  } else {
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) {
+      const int c = (sl + rot) & 3;
+      const uint64_t ctr = (idx0 + (uint64_t)(c * 8)) >> 2;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint64_t cc = ctr + h;
+        const uint4 r = philox4x32_10(make_uint4((uint32_t)cc, (uint32_t)(cc >> 32), 0u, 0u), sk0, sk1);
+        const int i0 = sl * 8 + h * 4;
+        const float2 v0 = mul2(make_float2(y[i0], y[i0 + 1]), inv2);
+        const float2 v1 = mul2(make_float2(y[i0 + 2], y[i0 + 3]), inv2);
+        qw[sl * 2 + h] = cvt_e4m3x4_rn(sr_e4m3_grid(v0.x, r.x), sr_e4m3_grid(v0.y, r.y),
+                                       sr_e4m3_grid(v1.x, r.z), sr_e4m3_grid(v1.y, r.w));
+      }
+    }
+  }
+  return (uint8_t)(e + 127);
+}
 
+// Store a block's codes: slot j holds chunk (j + rot) & 3, whose 8 codes go to
+// bytes 8 * chunk .. 8 * chunk + 7 of the block (four 8-byte stores; the
+// sectors fill up across the four).
+__device__ __forceinline__ void store_codes(uint8_t* qp, const uint32_t (&qw)[8], int rot) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    asm volatile("st.global.cs.v2.b32 [%0], {%1, %2};" ::"l"(qp + ((j + rot) & 3) * 8),
+                 "r"(qw[2 * j]), "r"(qw[2 * j + 1])
+                 : "memory");
+}
+
+// gamma for slot j of block k as 8 floats (in the order of the slot's words).
+__device__ __forceinline__ void gamma_slot(const uint8_t* smem, const FwdCfg& C, int j, int k,
+                                           float2 (&g)[4]) {
+  if (C.gamma_f32) {
+    const float4 lo = *reinterpret_cast<const float4*>(smem + ((size_t)(2 * j) * C.K + k) * 16);
+    const float4 hi = *reinterpret_cast<const float4*>(smem + ((size_t)(2 * j + 1) * C.K + k) * 16);
+    g[0] = make_float2(lo.x, lo.y); g[1] = make_float2(lo.z, lo.w);
+    g[2] = make_float2(hi.x, hi.y); g[3] = make_float2(hi.z, hi.w);
+  } else {
+    const uint4 v = *reinterpret_cast<const uint4*>(smem + ((size_t)j * C.K + k) * 16);
+    g[0] = bf16x2_to_f2(v.x); g[1] = bf16x2_to_f2(v.y);
+    g[2] = bf16x2_to_f2(v.z); g[3] = bf16x2_to_f2(v.w);
+  }
+}
+
+// TPR: threads per row as a compile-time constant (32, 64, 128, 256), or 0
+// for rows of fewer than 32 blocks, where C.tpr (< 32) rows share a warp.
+template <int MODE, int BPT, int TPR, bool SR>
+__global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const FwdArgs A, const FwdCfg C) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tpr = TPR ? TPR : C.tpr;
+  const int gthreads = TPR ? TPR : 32;
   const int tid = threadIdx.x;
-  constexpr int ncons = NCT;
-  if (tid == 0) {
+  const int g = tid / gthreads;             // row group within the CTA
+  const int t = tid - g * gthreads;         // thread within the group
+  const int rs = TPR ? 0 : (t >> C.log2_tpr);  // row slot within the stage (rps > 1 only)
+  const int tg = t & (tpr - 1);             // thread within the row
+  const int lane = tid & 31;
+  const int wig = t >> 5;                   // warp within the group
+  const int n_gwarps = gthreads >> 5;
+  const bool issuer = (t == 0);
+
+  uint8_t* ring = smem + C.ring_off + (size_t)g * C.stages * C.stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C.bar_off) + (size_t)g * 2 * C.stages;
+  uint64_t* empty = full + C.stages;
+  float2* red = reinterpret_cast<float2*>(smem + C.red_off) + (size_t)g * 2 * kRedSlots;
+  const bool has_gamma = (MODE != kModeCast) && (A.gamma != nullptr);
+
+  if (issuer) {
     for (int s = 0; s < C.stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], C.n_cwarps);
+      mbar_init(&empty[s], n_gwarps);
     }
     fence_barrier_init();
   }
+  // gamma -> shared memory in slot order, so that a warp's 16-byte reads of
+  // slot j fall on consecutive words: as fp32, half h of slot j of block k
+  // at ((2j + h) * K + k) * 16; as bf16 (long rows), slot j at (j * K + k) * 16.
+  if (has_gamma) {
+    for (int i = tid; i < C.K * 4; i += blockDim.x) {
+      const int k = i >> 2, j = i & 3;
+      const int c = (j + (k >> 1)) & 3;
+      const uint4 v = ldg128_nc(A.gamma + (size_t)k * kBlock + c * 8);
+      if (C.gamma_f32) {
+        const float4 lo = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
+        const float4 hi = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
+        *reinterpret_cast<float4*>(smem + ((size_t)(2 * j) * C.K + k) * 16) = lo;
+        *reinterpret_cast<float4*>(smem + ((size_t)(2 * j + 1) * C.K + k) * 16) = hi;
+      } else {
+        *reinterpret_cast<uint4*>(smem + ((size_t)j * C.K + k) * 16) = v;
+      }
+    }
+  }
   __syncthreads();
 
-  if (tid >= ncons) {
-    if (tid == ncons) produce_rows(A.x, C, stage0, full, empty, A.status);
-    return;
-  }
-
-  const int lane = tid & 31;
-  const int grp = tid >> C.log2_tpr;
-  const int tg = tid & (C.tpr - 1);
-  const bool has_gamma = (MODE != kModeCast) && (A.gamma != nullptr);
-
-  // gamma for this thread's blocks, in the same rotated chunk order as x.
-  uint32_t gw[BPT][16];
-#pragma unroll
-  for (int b = 0; b < BPT; ++b) {
-    const int k = tg + b * C.tpr;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint4 v = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // 1.0
-      if (has_gamma && k < C.K) {
-        const int c = (j + (k >> 1)) & 3;
-        v = ldg128_nc(A.gamma + (size_t)k * kBlock + c * 8);
-      }
-      gw[b][4 * j] = v.x; gw[b][4 * j + 1] = v.y; gw[b][4 * j + 2] = v.z; gw[b][4 * j + 3] = v.w;
+  // Global row group, numbered group-major so that the groups that get one
+  // more row block than the others are spread over all SMs.
+  const int64_t gg = (int64_t)g * gridDim.x + blockIdx.x;
+  const uint64_t pol = policy_evict_first();
+  if (issuer) {
+    for (int s = 0; s < C.stages; ++s) {
+      const int64_t rb = gg + (int64_t)s * C.ngt;
+      if (rb < C.n_row_blocks) issue_row_block(A.x, C, rb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
     }
   }
 
-  // A wait that gives up marks the kernel failed; the thread then keeps
-  // running (without waiting again) so that every named barrier of its row
-  // still completes, and its outputs are garbage but in bounds.
+  // A wait that gives up marks the kernel failed; threads then keep going
+  // without waiting so every named barrier still completes (outputs garbage,
+  // accesses in bounds).
   bool ok = true;
   int par = 0;
+  const int bar_id = 1 + g;
+  const int rot = (tg >> 1) & 3;           // the same for every block of the thread
   int64_t it = 0;
-  for (int64_t rb = blockIdx.x; rb < C.n_row_blocks; rb += gridDim.x, ++it, par ^= 1) {
+  for (int64_t rb = gg; rb < C.n_row_blocks; rb += C.ngt, ++it, par ^= 1) {
     const int s = (int)(it % C.stages);
     const uint32_t ph = (uint32_t)((it / C.stages) & 1);
     if (ok) ok = mbar_wait_bounded(&full[s], ph, A.status);
-
-    const int64_t row = rb * C.rps + grp;
+    const int64_t row = rb * C.rps + rs;
     const bool valid = row < C.T;
-    const uint32_t srow = smem_u32(stage0 + (size_t)s * C.stage_bytes + (size_t)grp * C.row_bytes);
+    const uint32_t srow = smem_u32(ring + (size_t)s * C.stage_bytes + (size_t)rs * C.row_bytes);
 
-    uint32_t xw[BPT][16];
-#pragma unroll
-    for (int b = 0; b < BPT; ++b) {
-      const int k = tg + b * C.tpr;
-      const bool have = valid && k < C.K;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (have) v = lds128(srow + (uint32_t)k * 64u + (uint32_t)(((j + (k >> 1)) & 3) * 16));
-        xw[b][4 * j] = v.x; xw[b][4 * j + 1] = v.y; xw[b][4 * j + 2] = v.z; xw[b][4 * j + 3] = v.w;
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-
-    if constexpr (MODE == kModeRMSNorm) {
-      // ---------------------------------------------------------- RMSNorm
-      float ss = 0.0f;
-#pragma unroll
-      for (int b = 0; b < BPT; ++b)
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float x0 = bf16lo(xw[b][j]), x1 = bf16hi(xw[b][j]);
-          ss = fmaf(x0, x0, ss);
-          ss = fmaf(x1, x1, ss);
-        }
-      ss = row_sum(ss, C, red, grp, tg, lane, par);
-      const float rinv = 1.0f / sqrtf(ss / (float)C.D + A.eps);
+    // ---- the row into registers, then the stage goes straight back to the
+    // issuer, so the copy of row block rb + stages * ngt overlaps this row's
+    // arithmetic (look-ahead = `stages` rows of compute).
+    // (RMSNorm keeps the row in the stage instead: it reads it twice and hands
+    // the stage back after its second pass, which needs far fewer registers.)
+    constexpr bool kHold = (MODE != kModeRMSNorm);
+    constexpr int kHoldB = kHold ? BPT : 1;
+    uint32_t xr[kHoldB][16];
+    if constexpr (kHold) {
 #pragma unroll
       for (int b = 0; b < BPT; ++b) {
-        const int k = tg + b * C.tpr;
+        const int k = tg + b * tpr;
+        const bool have = valid && k < C.K;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (have) v = lds128(srow + (uint32_t)k * 64u + (uint32_t)(((j + rot) & 3) * 16));
+          xr[b][4 * j] = v.x; xr[b][4 * j + 1] = v.y; xr[b][4 * j + 2] = v.z; xr[b][4 * j + 3] = v.w;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (issuer) {
+        const int64_t nrb = rb + (int64_t)C.stages * C.ngt;
+        if (nrb < C.n_row_blocks) {
+          if (ok) ok = mbar_wait_bounded(&empty[s], ph, A.status);
+          if (ok) issue_row_block(A.x, C, nrb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
+        }
+      }
+    }
+
+    // ---- pass 1: block maxima (MXNorm, Cast) or sum of squares (RMSNorm)
+    uint32_t mb[BPT];
+    float2 ss2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int b = 0; b < BPT; ++b) {
+      if constexpr (MODE == kModeRMSNorm) {
+        mb[b] = 0;
+        const int k = tg + b * tpr;
+        if (valid && k < C.K) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 v = lds128(srow + (uint32_t)k * 64u + (uint32_t)(((j + rot) & 3) * 16));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 xv = bf16x2_to_f2(w[i]);
+              ss2 = fma2(xv, xv, ss2);
+            }
+          }
+        }
+      } else {
+        mb[b] = block_absmax16(xr[b]);
+      }
+    }
+
+    float2* redp = red + par * kRedSlots;
+    if constexpr (MODE == kModeRMSNorm) {
+      // ---------------------------------------------------------- RMSNorm
+      const float ss = row_sum<TPR>(ss2.x + ss2.y, C, redp, bar_id, wig, lane);
+      const float rinv = 1.0f / sqrtf(ss / (float)C.D + A.eps);
+      const float2 r2 = make_float2(rinv, rinv);
+#pragma unroll
+      for (int b = 0; b < BPT; ++b) {
+        const int k = tg + b * tpr;
         if (!valid || k >= C.K) continue;
-        const int rot = (k >> 1) & 3;
         uint16_t* yrow = A.y + row * (int64_t)C.D + (int64_t)k * kBlock;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
+          const uint4 v = lds128(srow + (uint32_t)k * 64u + (uint32_t)(((j + rot) & 3) * 16));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          float2 gf[4];
+          if (has_gamma) gamma_slot(smem, C, j, k, gf);
           uint32_t o[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const uint32_t w = xw[b][4 * j + i], g = gw[b][4 * j + i];
-            float y0 = __fmul_rn(bf16lo(w), rinv), y1 = __fmul_rn(bf16hi(w), rinv);
-            if (has_gamma) { y0 = __fmul_rn(y0, bf16lo(g)); y1 = __fmul_rn(y1, bf16hi(g)); }
-            const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+            float2 yv = mul2(bf16x2_to_f2(w[i]), r2);
+            if (has_gamma) yv = mul2(yv, gf[i]);
+            const __nv_bfloat162 h = __floats2bfloat162_rn(yv.x, yv.y);
             o[i] = *reinterpret_cast<const uint32_t*>(&h);
           }
           stg128_stream(yrow + ((j + rot) & 3) * 8, make_uint4(o[0], o[1], o[2], o[3]));
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (issuer) {
+        const int64_t nrb = rb + (int64_t)C.stages * C.ngt;
+        if (nrb < C.n_row_blocks) {
+          if (ok) ok = mbar_wait_bounded(&empty[s], ph, A.status);
+          if (ok) issue_row_block(A.x, C, nrb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
+        }
+      }
     } else {
       // ------------------------------------------------- MXNorm / MXCast
-      uint32_t mb[BPT];
-#pragma unroll
-      for (int b = 0; b < BPT; ++b) mb[b] = absmax_bits_bf16x2(xw[b], 16);
-      float sc = 1.0f, G = 0.0f;
+      float sc = 1.0f;
       if constexpr (MODE == kModeMXNorm) {
-        G = row_pmean<BPT>(mb, A, C, red, grp, tg, lane, par);
+        const float G = row_pmean<BPT, TPR>(mb, A, C, redp, bar_id, wig, lane);
         sc = (G == 0.0f) ? 0.0f : __frcp_rn(G);
         if (valid && tg == 0 && A.G_out) A.G_out[row] = G;
       }
+      const float2 s2 = make_float2(sc, sc);
 #pragma unroll
       for (int b = 0; b < BPT; ++b) {
-        const int k = tg + b * C.tpr;
+        const int k = tg + b * tpr;
         if (!valid || k >= C.K) continue;
-        const int rot = (k >> 1) & 3;
         float y[32];
         float a;
         if (MODE == kModeMXNorm && has_gamma) {
-          a = 0.0f;
+          float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            y[2 * j] = __fmul_rn(__fmul_rn(bf16lo(xw[b][j]), sc), bf16lo(gw[b][j]));
-            y[2 * j + 1] = __fmul_rn(__fmul_rn(bf16hi(xw[b][j]), sc), bf16hi(gw[b][j]));
-            a = max_abs_nan(a, y[2 * j]);
-            a = max_abs_nan(a, y[2 * j + 1]);
-          }
-        } else if (MODE == kModeMXNorm) {
+          for (int j = 0; j < 4; ++j) {
+            float2 gf[4];
+            gamma_slot(smem, C, j, k, gf);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            y[2 * j] = __fmul_rn(bf16lo(xw[b][j]), sc);
-            y[2 * j + 1] = __fmul_rn(bf16hi(xw[b][j]), sc);
+            for (int i = 0; i < 4; ++i) {
+              const float2 yv = mul2(mul2(bf16x2_to_f2(xr[b][4 * j + i]), s2), gf[i]);
+              y[8 * j + 2 * i] = yv.x;
+              y[8 * j + 2 * i + 1] = yv.y;
+              if (i & 1) a1 = max3_abs_nan(a1, yv.x, yv.y);
+              else a0 = max3_abs_nan(a0, yv.x, yv.y);
+            }
           }
-          a = __fmul_rn(bf16bits_to_float(mb[b]), sc);  // rounding is monotone
+          a = max3_abs_nan(a0, a1, 0.0f);
         } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            y[2 * j] = bf16lo(xw[b][j]);
-            y[2 * j + 1] = bf16hi(xw[b][j]);
+          for (int w = 0; w < 16; ++w) {
+            float2 yv = bf16x2_to_f2(xr[b][w]);
+            if (MODE == kModeMXNorm) yv = mul2(yv, s2);
+            y[2 * w] = yv.x;
+            y[2 * w + 1] = yv.y;
           }
-          a = bf16bits_to_float(mb[b]);
+          // fl(m * s) is the block max of fl(x * s): rounding is monotone.
+          a = (MODE == kModeMXNorm) ? __fmul_rn(bf16bits_to_float(mb[b]), sc) : bf16bits_to_float(mb[b]);
         }
-        const int e = e8m0_exponent_bits(__float_as_uint(a) & 0x7FFFFFFFu);  // a >= 0 or NaN
         uint32_t qw[8];
-        uint8_t code;
-        if (e == 128) {
-          code = 0xFF;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) qw[i] = 0x7F7F7F7Fu;
-        } else {
-          code = (uint8_t)(e + 127);
-          const float inv = exp2_int(-e);
-          if constexpr (!SR) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint32_t lo = cvt_e4m3x2_rn(__fmul_rn(y[4 * i], inv), __fmul_rn(y[4 * i + 1], inv));
-              const uint32_t hi = cvt_e4m3x2_rn(__fmul_rn(y[4 * i + 2], inv), __fmul_rn(y[4 * i + 3], inv));
-              qw[i] = lo | (hi << 16);
-            }
-          } else {
-#pragma unroll
-            for (int sl = 0; sl < 4; ++sl) {
-              const int c = (sl + rot) & 3;  // chunk held in slot sl
-              const uint64_t ctr = (uint64_t)(row * (int64_t)C.D + (int64_t)k * kBlock + c * 8) >> 2;
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const uint64_t cc = ctr + h;
-                const uint4 r = philox4x32_10(make_uint4((uint32_t)cc, (uint32_t)(cc >> 32), 0u, 0u),
-                                              A.seed_lo, A.seed_hi);
-                const int i0 = sl * 8 + h * 4;
-                const float v0 = sr_e4m3_grid(__fmul_rn(y[i0], inv), r.x);
-                const float v1 = sr_e4m3_grid(__fmul_rn(y[i0 + 1], inv), r.y);
-                const float v2 = sr_e4m3_grid(__fmul_rn(y[i0 + 2], inv), r.z);
-                const float v3 = sr_e4m3_grid(__fmul_rn(y[i0 + 3], inv), r.w);
-                qw[sl * 2 + h] = cvt_e4m3x2_rn(v0, v1) | (cvt_e4m3x2_rn(v2, v3) << 16);
-              }
-            }
-          }
-        }
-        // Slot sl holds chunk (sl + rot) & 3; put chunk c at word pair 2c.
-        // Two select stages rotate by (rot & 1) and then by (rot & 2) slots.
-        uint32_t o[8];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) o[2 * c + h] = (rot & 1) ? qw[2 * ((c + 3) & 3) + h] : qw[2 * c + h];
-        uint32_t o2[8];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) o2[2 * c + h] = (rot & 2) ? o[2 * ((c + 2) & 3) + h] : o[2 * c + h];
-        uint8_t* qp = A.q + row * (int64_t)C.D + (int64_t)k * kBlock;
-        stg128_stream(qp, make_uint4(o2[0], o2[1], o2[2], o2[3]));
-        stg128_stream(qp + 16, make_uint4(o2[4], o2[5], o2[6], o2[7]));
+        const uint64_t idx0 = (uint64_t)(row * (int64_t)C.D + (int64_t)k * kBlock);
+        const uint8_t code = quantise_block<SR>(y, a, rot, idx0, A.seed_lo, A.seed_hi, qw);
+        store_codes(A.q + row * (int64_t)C.D + (int64_t)k * kBlock, qw, rot);
         if (A.scale_mma) A.scales[mma_scale_offset(row, k, A.kp4)] = code;
         else A.scales[row * (int64_t)C.K + k] = code;
       }
+    }
+
+  }
+  // Leave no copy in flight: the issuer waits for the last phase of every stage
+  // it filled (already complete unless a wait gave up above).
+  if (issuer && !ok) {
+    for (int s = 0; s < C.stages; ++s) {
+      const int64_t last_it = it - 1 - ((it - 1 - s) % C.stages + C.stages) % C.stages;
+      if (last_it >= 0) mbar_wait_bounded(&full[s], (uint32_t)((last_it / C.stages) & 1), A.status);
     }
   }
 }

@@ -102,8 +102,9 @@ def test_other_entry_points_validate(L):
 
 
 def test_tuning_validation(L):
-    assert L.mxnorm_set_tuning(96, 0, 0) == ops.MXN_ERR_ARG
-    assert L.mxnorm_set_tuning(0, 1, 0) == ops.MXN_ERR_ARG
+    assert L.mxnorm_set_tuning(100, 0, 0) == ops.MXN_ERR_ARG
+    assert L.mxnorm_set_tuning(1024, 0, 0) == ops.MXN_ERR_ARG
+    assert L.mxnorm_set_tuning(0, 17, 0) == ops.MXN_ERR_ARG
     assert L.mxnorm_set_tuning(0, 0, 9) == ops.MXN_ERR_ARG
     assert L.mxnorm_set_tuning(256, 4, 2) == ops.MXN_OK
     assert L.mxnorm_set_tuning(0, 0, 0) == ops.MXN_OK
