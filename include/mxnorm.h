@@ -159,6 +159,29 @@ int mxnorm_bwd(const void* x, const void* dy, const void* gamma, const float* G,
 /* Scratch bytes mxnorm_bwd needs for (T, D) on the current device. */
 size_t mxnorm_bwd_workspace_size(int64_t T, int64_t D);
 
+/*
+ * mxnorm_bwd without a workspace argument, for callers that cannot allocate
+ * device memory when they call: code recorded into a CUDA graph whose memory
+ * plan is fixed up front, plugins inside an engine that owns every allocation,
+ * and real-time loops that must not call cudaMalloc.  The paper has no
+ * counterpart; this is a deployment convenience.
+ *
+ * Same arguments, results and limits as mxnorm_bwd (D <= 16384), except that
+ * the dgamma partial sums live in one 8 MiB scratch array inside this library
+ * (2^21 fp32, allocated when a device loads the library, held until exit).
+ * The call allocates nothing.  To fit the scratch it may launch fewer CTAs
+ * than mxnorm_bwd (at most 2^21 / (rows per stage * D) of them); it returns
+ * MXN_ERR_UNSUPPORTED if even one CTA's partial rows would not fit.
+ * The first call on a device looks up the scratch array's device address
+ * (cudaGetSymbolAddress); make that first call outside any stream capture.
+ * Every call on a device shares the one scratch array: calls that may overlap
+ * on the GPU (different streams, or different host threads) race and must be
+ * serialised by the caller.  Each call overwrites every partial it reads, so
+ * nothing has to be cleared between calls.
+ */
+int mxnorm_bwd_noalloc(const void* x, const void* dy, const void* gamma, const float* G,
+                       void* dx, void* dgamma, int64_t T, int64_t D, void* stream);
+
 /* Message for the last error on the calling thread ("" if none).  The string
    stays valid until the thread's next call into the library. */
 const char* mxnorm_last_error(void);

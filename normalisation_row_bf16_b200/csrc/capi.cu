@@ -372,6 +372,35 @@ int plan_bwd(int64_t T, int D, int sms, Plan* P) {
   return plan_rows(T, D, D, 2, bwd_kernel, sms, P);
 }
 
+// ----------------------------------------------- allocation-free backward
+//
+// Scratch for mxnorm_bwd_noalloc: the per-CTA dgamma partial sums, 2^21 fp32
+// (8 MiB).  Every device that loads this library holds it until the process
+// exits.  In host code the name is only a host-side stand-in; its device
+// address comes from cudaGetSymbolAddress, looked up once per device with
+// that device current.
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 21;
+static __device__ __align__(256) float g_bwd_noalloc_scratch[kNoAllocScratchFloats];
+
+float* g_noalloc_scratch_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+int noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MXN_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_bwd_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(noalloc scratch)");
+    g_noalloc_scratch_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_scratch_ptr[dev];
+  return MXN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -516,6 +545,56 @@ int mxnorm_bwd(const void* x, const void* dy, const void* gamma, const float* G,
   if (dgamma) {
     dgamma_reduce_kernel<<<(unsigned)((D + 31) / 32), dim3(32, 32), 0, s>>>(
         A.partial, (int64_t)P.grid * P.C.rps, (int)D, static_cast<uint16_t*>(dgamma));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "dgamma_reduce_kernel launch");
+  }
+  return MXN_OK;
+}
+
+int mxnorm_bwd_noalloc(const void* x, const void* dy, const void* gamma, const float* G,
+                       void* dx, void* dgamma, int64_t T, int64_t D, void* stream) {
+  t_err.clear();
+  int rc = check_common(x, T, D, D);
+  if (!rc) rc = check_out(dy, "dy");
+  if (!rc) rc = check_out(G, "G");
+  if (!rc) rc = check_out(dx, "dx");
+  if (!rc) rc = check_opt(gamma, "gamma");
+  if (!rc) rc = check_opt(dgamma, "dgamma");
+  if (rc) return rc;
+  if (D > kMaxBwdD) return fail(MXN_ERR_UNSUPPORTED, "mxnorm_bwd_noalloc: D = %lld > %d", (long long)D, kMaxBwdD);
+  if (dgamma && !gamma) return fail(MXN_ERR_ARG, "dgamma requested without gamma");
+  if ((rc = injected())) return rc;
+  if (T == 0) return MXN_OK;
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  Plan P;
+  if ((rc = plan_bwd(T, (int)D, dev.sms, &P))) return rc;
+  float* scratch = nullptr;
+  if (dgamma) {
+    if ((rc = noalloc_scratch(&scratch))) return rc;
+    // Each CTA writes rps partial rows of D floats: launch no more CTAs than
+    // the scratch holds (the kernel is persistent, so fewer CTAs cover all rows).
+    const int64_t per_cta = (int64_t)P.C.rps * D;
+    const int64_t max_ctas = (int64_t)kNoAllocScratchFloats / per_cta;
+    if (max_ctas < 1)
+      return fail(MXN_ERR_UNSUPPORTED,
+                  "mxnorm_bwd_noalloc: %lld partial floats per CTA exceed the %zu-float scratch",
+                  (long long)per_cta, kNoAllocScratchFloats);
+    if (P.grid > max_ctas) P.grid = (int)max_ctas;
+  }
+  BwdArgs A{};
+  A.x = static_cast<const uint16_t*>(x);
+  A.dy = static_cast<const uint16_t*>(dy);
+  A.gamma = static_cast<const uint16_t*>(gamma);
+  A.G = G;
+  A.dx = static_cast<uint16_t*>(dx);
+  A.partial = scratch;
+  A.status = dev.status;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = launch(P, &A, s))) return rc;
+  if (dgamma) {
+    dgamma_reduce_kernel<<<(unsigned)((D + 31) / 32), dim3(32, 32), 0, s>>>(
+        scratch, (int64_t)P.grid * P.C.rps, (int)D, static_cast<uint16_t*>(dgamma));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "dgamma_reduce_kernel launch");
   }

@@ -30,6 +30,7 @@ SIGNATURES = {
     "rmsnorm_then_mxcast": (_I32, [_P, _P, _F32, _P, _P, _P, _I64, _I64, _I64, _I32, _P]),
     "mxnorm_bwd": (_I32, [_P, _P, _P, _P, _P, _P, _I64, _I64, _P, _SZ, _P]),
     "mxnorm_bwd_workspace_size": (_SZ, [_I64, _I64]),
+    "mxnorm_bwd_noalloc": (_I32, [_P, _P, _P, _P, _P, _P, _I64, _I64, _P]),
     "mxnorm_last_error": (ctypes.c_char_p, []),
     "mxnorm_device_status": (_I32, [_P]),
     "mxnorm_set_tuning": (_I32, [_I32, _I32, _I32]),
@@ -177,6 +178,24 @@ def mxnorm_bwd(x, dy, gamma, G, dx=None, dgamma=None, workspace=None, want_dgamm
         nbytes = workspace.numel() * workspace.element_size()
     _check(lib().mxnorm_bwd(_ptr(x), _ptr(dy), _ptr(gamma), _ptr(G), _ptr(dx), _ptr(dgamma), T, D,
                             _ptr(workspace), nbytes, _stream(stream)))
+    return dx, dgamma
+
+
+def mxnorm_bwd_noalloc(x, dy, gamma, G, dx=None, dgamma=None, want_dgamma: bool = True,
+                       stream=None):
+    """The backward through the entry point that allocates no device memory
+    (its dgamma partials live in the library's own scratch array; calls that
+    overlap on the GPU race).  Outputs are allocated here only when not given."""
+    T, D, ld = _rows_ld(x)
+    if ld != D or dy.shape != x.shape or not dy.is_contiguous() or dy.dtype != torch.bfloat16:
+        raise ValueError("x and dy must be dense bf16 [T, D]")
+    gamma = _bf16_vec(gamma, D)
+    if dx is None:
+        dx = torch.empty_like(x)
+    if gamma is not None and want_dgamma and dgamma is None:
+        dgamma = torch.empty(D, dtype=torch.bfloat16, device=x.device)
+    _check(lib().mxnorm_bwd_noalloc(_ptr(x), _ptr(dy), _ptr(gamma), _ptr(G), _ptr(dx), _ptr(dgamma),
+                                    T, D, _stream(stream)))
     return dx, dgamma
 
 

@@ -1,0 +1,54 @@
+"""The allocation-free backward entry point, mxnorm_bwd_noalloc.
+
+It serves callers that cannot allocate device memory at call time (code
+captured into a CUDA graph with a fixed memory plan, engines that own every
+allocation, real-time loops).  It must give the same dx and dgamma as
+mxnorm_bwd with a caller-provided workspace, within the backward's tolerance,
+on two calls in a row (the second call reuses the library's scratch array as
+the first left it).  This file runs last so that a failure here leaves every
+other test already run.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from normalisation_row_bf16_b200 import build as nbuild
+from normalisation_row_bf16_b200 import ops, synthetic
+
+from parity_util import BWD_RTOL_L2, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _call_noalloc(x, dy, g, G, dx, dg):
+    """Straight through the C ABI: no workspace argument exists."""
+    L = ops.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = L.mxnorm_bwd_noalloc(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(dy.data_ptr()),
+                              ctypes.c_void_p(g.data_ptr()), ctypes.c_void_p(G.data_ptr()),
+                              ctypes.c_void_p(dx.data_ptr()), ctypes.c_void_p(dg.data_ptr()),
+                              x.shape[0], x.shape[1], stream)
+    assert rc == ops.MXN_OK, L.mxnorm_last_error().decode()
+
+
+@pytest.mark.parametrize("T,D", [(8192, 4096), (300, 1024), (64, 16384)])
+def test_noalloc_backward_matches_workspace_backward(T, D):
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    nbuild.build()
+    x = synthetic.activations(T, D, "normal", seed=D, device="cuda")
+    g = synthetic.gamma(D, seed=D, device="cuda")
+    _, _, G = ops.mxnorm_fwd(x, g, 2.0)
+    for call in range(2):
+        dy = synthetic.upstream_grad(T, D, seed=D + call, device="cuda")
+        dx_ref, dg_ref = ops.mxnorm_bwd(x, dy, g, G)
+        dx = torch.full_like(x, float("nan"))
+        dg = torch.full((D,), float("nan"), dtype=torch.bfloat16, device="cuda")
+        _call_noalloc(x, dy, g, G, dx, dg)
+        torch.cuda.synchronize()
+        assert rel_l2(dx.float().cpu().numpy(), dx_ref.float().cpu().numpy()) <= BWD_RTOL_L2
+        assert rel_l2(dg.float().cpu().numpy(), dg_ref.float().cpu().numpy()) <= BWD_RTOL_L2
+        assert torch.isfinite(dg.float()).all()
+    assert ops.device_status() == ops.MXN_OK
