@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmxnorm_b200.so")
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
-              "-Xcompiler", "-fPIC", "-shared", "-Xptxas", "-warn-spills"]
+              "-Xcompiler", "-fPIC", "-Xptxas", "-warn-spills"]
 
 
 def sources():
@@ -38,15 +38,31 @@ def nvcc() -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every translation unit in csrc/ (in parallel) and link the library."""
     if not force and not is_stale():
         return LIB
     tus = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    procs = []
+    for tu in tus:
+        obj = os.path.join(objdir, os.path.basename(tu) + f".{os.getpid()}.o")
+        cmd = [nvcc(), *NVCC_FLAGS, "-c", "-I" + INCLUDE, "-o", obj, tu]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        procs.append((obj, subprocess.Popen(cmd)))
+    objs = []
+    failed = False
+    for obj, p in procs:
+        failed |= p.wait() != 0
+        objs.append(obj)
+    if failed:
+        raise RuntimeError("nvcc failed")
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I" + INCLUDE, "-o", tmp, *tus]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
+    subprocess.run([nvcc(), "-shared", "-o", tmp, *objs], check=True)
     os.replace(tmp, LIB)
+    for o in objs:
+        os.remove(o)
     return LIB
 
 

@@ -8,6 +8,7 @@
 #include <string>
 #include <tuple>
 
+#include "fwd_dispatch.h"
 #include "mxnorm.h"
 #include "row_bwd.cuh"
 #include "row_fwd.cuh"
@@ -221,25 +222,12 @@ int check_opt(const void* p, const char* name) {
   return MXN_OK;
 }
 
-// The instantiation for (blocks per thread, threads per row): 32 threads per
-// row for up to 4 blocks each (D <= 4096), 64..256 threads with 4 blocks each
-// beyond, a runtime segment width below 32 blocks per row.
-template <int MODE, bool SR>
-const void* fwd_kernel(int bpt, int tpr) {
-  if (tpr < 32) return bpt == 1 ? (const void*)row_fwd_kernel<MODE, 1, 0, SR> : nullptr;
-  if (tpr == 32) {
-    switch (bpt) {
-      case 1: return (const void*)row_fwd_kernel<MODE, 1, 32, SR>;
-      case 2: return (const void*)row_fwd_kernel<MODE, 2, 32, SR>;
-      case 4: return (const void*)row_fwd_kernel<MODE, 4, 32, SR>;
-      default: return nullptr;
-    }
-  }
-  if (bpt != 4) return nullptr;
-  switch (tpr) {
-    case 64: return (const void*)row_fwd_kernel<MODE, 4, 64, SR>;
-    case 128: return (const void*)row_fwd_kernel<MODE, 4, 128, SR>;
-    case 256: return (const void*)row_fwd_kernel<MODE, 4, 256, SR>;
+const void* fwd_kernel(int mode, bool sr, bool has_gamma, int bpt, int tpr) {
+  switch (mode) {
+    case kModeMXNorm:
+      return sr ? fwd_kernel_mxnorm_sr(bpt, tpr, has_gamma) : fwd_kernel_mxnorm_rne(bpt, tpr, has_gamma);
+    case kModeCast: return fwd_kernel_cast(bpt, tpr, sr);
+    case kModeRMSNorm: return fwd_kernel_rmsnorm(bpt, tpr, has_gamma);
     default: return nullptr;
   }
 }
@@ -284,8 +272,8 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int64_t T, int D, int64_t ld_x,
     int st = (int)((176u * 1024u) / ((size_t)gmax * C.rps * 2u * (uint32_t)D));
     C.stages = st < 1 ? 1 : (st > 3 ? 3 : st);
   }
-  C.gamma_f32 = D <= 8192 ? 1 : 0;
-  C.gamma_bytes = gamma_smem ? (uint32_t)align_up((C.gamma_f32 ? 4u : 2u) * (uint32_t)D, 128) : 0u;
+  // gamma in shared memory: fp32 for up to 64 threads per row (D <= 8192), else bf16
+  C.gamma_bytes = gamma_smem ? (uint32_t)align_up((gamma_fp32(C.tpr) ? 4u : 2u) * (uint32_t)D, 128) : 0u;
   const size_t per_group = (size_t)C.stages * C.stage_bytes;
   // Shared memory per group: its ring, its 2 * stages barriers and its two
   // reduction slot arrays; plus gamma and 16 bytes of alignment once.
@@ -313,11 +301,7 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int64_t T, int D, int64_t ld_x,
   C.red_off = C.bar_off + (uint32_t)(ng * 2 * C.stages * sizeof(uint64_t));
   P->smem = C.red_off + (size_t)ng * 2 * kRedSlots * sizeof(float2);
   P->threads = ng * C.gthreads;
-  P->kernel = sr ? (mode == kModeMXNorm ? fwd_kernel<kModeMXNorm, true>(bpt, C.tpr)
-                                        : fwd_kernel<kModeCast, true>(bpt, C.tpr))
-                 : (mode == kModeMXNorm ? fwd_kernel<kModeMXNorm, false>(bpt, C.tpr)
-                    : mode == kModeCast ? fwd_kernel<kModeCast, false>(bpt, C.tpr)
-                                        : fwd_kernel<kModeRMSNorm, false>(bpt, C.tpr));
+  P->kernel = fwd_kernel(mode, sr, gamma_smem, bpt, C.tpr);
   if (!P->kernel) return fail(MXN_ERR_UNSUPPORTED, "no kernel for D = %d", D);
   int occ = 0;
   int rc = occupancy(P->kernel, P->threads, P->smem, &occ);

@@ -42,7 +42,7 @@ enum PMode { kP1 = 1, kP2 = 2, kP4 = 4, kPInf = 0, kPGeneral = 3 };
 // Threads per CTA the register budget is sized for: a thread holding 4 blocks
 // of its row needs ~120 registers (512 threads), 2 blocks ~96 (640), 1 block
 // fits in 80 (768).
-constexpr int fwd_max_threads(int bpt) { return bpt >= 4 ? 512 : (bpt == 2 ? 640 : 768); }
+__host__ __device__ constexpr int fwd_max_threads(int bpt) { return bpt >= 4 ? 512 : (bpt == 2 ? 640 : 768); }
 constexpr int kRedSlots = 16;  // warps per row group, at most
 
 struct FwdCfg {
@@ -59,7 +59,6 @@ struct FwdCfg {
   uint32_t row_bytes;    // 2 * D
   uint32_t stage_bytes;  // rps * row_bytes
   uint32_t gamma_bytes;  // shared-memory gamma (0 when unused)
-  int gamma_f32;         // gamma held as fp32 (else bf16) in shared memory
   uint32_t ring_off, bar_off, red_off;
 };
 
@@ -229,12 +228,9 @@ template <bool SR>
 __device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a, int rot,
                                                   uint64_t idx0, uint32_t sk0, uint32_t sk1,
                                                   uint32_t (&qw)[8]) {
-  const int e = e8m0_exponent_bits(__float_as_uint(a) & 0x7FFFFFFFu);
-  if (e == 128) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) qw[i] = 0x7F7F7F7Fu;
-    return 0xFF;
-  }
+  const int e_raw = e8m0_exponent_bits(__float_as_uint(a) & 0x7FFFFFFFu);
+  const bool nan_block = (e_raw == 128);     // NaN / inf in the block: codes 0x7F, scale 0xFF
+  const int e = nan_block ? 0 : e_raw;
   const float inv = exp2_int(-e);
   const float2 inv2 = make_float2(inv, inv);
   if constexpr (!SR) {
@@ -261,7 +257,9 @@ __device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a,
       }
     }
   }
-  return (uint8_t)(e + 127);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) qw[i] = nan_block ? 0x7F7F7F7Fu : qw[i];
+  return nan_block ? (uint8_t)0xFF : (uint8_t)(e + 127);
 }
 
 // Store a block's codes: slot j holds chunk (j + rot) & 3, whose 8 codes go to
@@ -276,23 +274,28 @@ __device__ __forceinline__ void store_codes(uint8_t* qp, const uint32_t (&qw)[8]
 }
 
 // gamma for slot j of block k as 8 floats (in the order of the slot's words).
-__device__ __forceinline__ void gamma_slot(const uint8_t* smem, const FwdCfg& C, int j, int k,
-                                           float2 (&g)[4]) {
-  if (C.gamma_f32) {
-    const float4 lo = *reinterpret_cast<const float4*>(smem + ((size_t)(2 * j) * C.K + k) * 16);
-    const float4 hi = *reinterpret_cast<const float4*>(smem + ((size_t)(2 * j + 1) * C.K + k) * 16);
+template <bool F32>
+__device__ __forceinline__ void gamma_slot(const uint8_t* smem, int K, int j, int k, float2 (&g)[4]) {
+  if constexpr (F32) {
+    const float4 lo = *reinterpret_cast<const float4*>(smem + ((size_t)(2 * j) * K + k) * 16);
+    const float4 hi = *reinterpret_cast<const float4*>(smem + ((size_t)(2 * j + 1) * K + k) * 16);
     g[0] = make_float2(lo.x, lo.y); g[1] = make_float2(lo.z, lo.w);
     g[2] = make_float2(hi.x, hi.y); g[3] = make_float2(hi.z, hi.w);
   } else {
-    const uint4 v = *reinterpret_cast<const uint4*>(smem + ((size_t)j * C.K + k) * 16);
+    const uint4 v = *reinterpret_cast<const uint4*>(smem + ((size_t)j * K + k) * 16);
     g[0] = bf16x2_to_f2(v.x); g[1] = bf16x2_to_f2(v.y);
     g[2] = bf16x2_to_f2(v.z); g[3] = bf16x2_to_f2(v.w);
   }
 }
 
+// gamma sits in shared memory as fp32 for rows of up to 8192 elements (up to
+// 64 threads per row), as bf16 beyond.
+__host__ __device__ constexpr bool gamma_fp32(int tpr) { return tpr == 0 || tpr <= 64; }
+
 // TPR: threads per row as a compile-time constant (32, 64, 128, 256), or 0
 // for rows of fewer than 32 blocks, where C.tpr (< 32) rows share a warp.
-template <int MODE, int BPT, int TPR, bool SR>
+// HG: gamma given (MXNorm, RMSNorm); its shared-memory format follows TPR.
+template <int MODE, int BPT, int TPR, bool SR, bool HG>
 __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const FwdArgs A, const FwdCfg C) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tpr = TPR ? TPR : C.tpr;
@@ -311,7 +314,8 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C.bar_off) + (size_t)g * 2 * C.stages;
   uint64_t* empty = full + C.stages;
   float2* red = reinterpret_cast<float2*>(smem + C.red_off) + (size_t)g * 2 * kRedSlots;
-  const bool has_gamma = (MODE != kModeCast) && (A.gamma != nullptr);
+  constexpr bool has_gamma = (MODE != kModeCast) && HG;
+  constexpr bool kGF32 = gamma_fp32(TPR);
 
   if (issuer) {
     for (int s = 0; s < C.stages; ++s) {
@@ -323,12 +327,12 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
   // gamma -> shared memory in slot order, so that a warp's 16-byte reads of
   // slot j fall on consecutive words: as fp32, half h of slot j of block k
   // at ((2j + h) * K + k) * 16; as bf16 (long rows), slot j at (j * K + k) * 16.
-  if (has_gamma) {
+  if constexpr (has_gamma) {
     for (int i = tid; i < C.K * 4; i += blockDim.x) {
       const int k = i >> 2, j = i & 3;
       const int c = (j + (k >> 1)) & 3;
       const uint4 v = ldg128_nc(A.gamma + (size_t)k * kBlock + c * 8);
-      if (C.gamma_f32) {
+      if constexpr (kGF32) {
         const float4 lo = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
         const float4 hi = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
         *reinterpret_cast<float4*>(smem + ((size_t)(2 * j) * C.K + k) * 16) = lo;
@@ -432,23 +436,24 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
 #pragma unroll
       for (int b = 0; b < BPT; ++b) {
         const int k = tg + b * tpr;
-        if (!valid || k >= C.K) continue;
+        const bool blk = valid && k < C.K;
+        const int kk = k < C.K ? k : C.K - 1;          // in-range smem reads
         uint16_t* yrow = A.y + row * (int64_t)C.D + (int64_t)k * kBlock;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint4 v = lds128(srow + (uint32_t)k * 64u + (uint32_t)(((j + rot) & 3) * 16));
+          const uint4 v = lds128(srow + (uint32_t)kk * 64u + (uint32_t)(((j + rot) & 3) * 16));
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
           float2 gf[4];
-          if (has_gamma) gamma_slot(smem, C, j, k, gf);
+          if constexpr (has_gamma) gamma_slot<kGF32>(smem, C.K, j, kk, gf);
           uint32_t o[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             float2 yv = mul2(bf16x2_to_f2(w[i]), r2);
-            if (has_gamma) yv = mul2(yv, gf[i]);
+            if constexpr (has_gamma) yv = mul2(yv, gf[i]);
             const __nv_bfloat162 h = __floats2bfloat162_rn(yv.x, yv.y);
             o[i] = *reinterpret_cast<const uint32_t*>(&h);
           }
-          stg128_stream(yrow + ((j + rot) & 3) * 8, make_uint4(o[0], o[1], o[2], o[3]));
+          if (blk) stg128_stream(yrow + ((j + rot) & 3) * 8, make_uint4(o[0], o[1], o[2], o[3]));
         }
       }
       __syncwarp();
@@ -472,15 +477,16 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
 #pragma unroll
       for (int b = 0; b < BPT; ++b) {
         const int k = tg + b * tpr;
-        if (!valid || k >= C.K) continue;
+        const bool blk = valid && k < C.K;             // blocks past K compute on zeros
+        const int kk = k < C.K ? k : C.K - 1;          // in-range gamma reads
         float y[32];
         float a;
-        if (MODE == kModeMXNorm && has_gamma) {
+        if constexpr (MODE == kModeMXNorm && has_gamma) {
           float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             float2 gf[4];
-            gamma_slot(smem, C, j, k, gf);
+            gamma_slot<kGF32>(smem, C.K, j, kk, gf);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float2 yv = mul2(mul2(bf16x2_to_f2(xr[b][4 * j + i]), s2), gf[i]);
@@ -505,9 +511,11 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
         uint32_t qw[8];
         const uint64_t idx0 = (uint64_t)(row * (int64_t)C.D + (int64_t)k * kBlock);
         const uint8_t code = quantise_block<SR>(y, a, rot, idx0, A.seed_lo, A.seed_hi, qw);
-        store_codes(A.q + row * (int64_t)C.D + (int64_t)k * kBlock, qw, rot);
-        if (A.scale_mma) A.scales[mma_scale_offset(row, k, A.kp4)] = code;
-        else A.scales[row * (int64_t)C.K + k] = code;
+        if (blk) {
+          store_codes(A.q + row * (int64_t)C.D + (int64_t)k * kBlock, qw, rot);
+          const int64_t so = A.scale_mma ? mma_scale_offset(row, k, A.kp4) : row * (int64_t)C.K + k;
+          A.scales[so] = code;
+        }
       }
     }
 
@@ -519,6 +527,30 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
       const int64_t last_it = it - 1 - ((it - 1 - s) % C.stages + C.stages) % C.stages;
       if (last_it >= 0) mbar_wait_bounded(&full[s], (uint32_t)((last_it / C.stages) & 1), A.status);
     }
+  }
+}
+
+// The instantiation for (blocks per thread, threads per row): 32 threads per
+// row for up to 4 blocks each (rows of up to 128 blocks), 64..256 threads with
+// 4 blocks each beyond, a runtime segment width for rows under 32 blocks.
+// Each translation unit that calls this instantiates its own mode's kernels.
+template <int MODE, bool SR, bool HG>
+const void* pick_fwd_shape(int bpt, int tpr) {
+  if (tpr < 32) return bpt == 1 ? (const void*)row_fwd_kernel<MODE, 1, 0, SR, HG> : nullptr;
+  if (tpr == 32) {
+    switch (bpt) {
+      case 1: return (const void*)row_fwd_kernel<MODE, 1, 32, SR, HG>;
+      case 2: return (const void*)row_fwd_kernel<MODE, 2, 32, SR, HG>;
+      case 4: return (const void*)row_fwd_kernel<MODE, 4, 32, SR, HG>;
+      default: return nullptr;
+    }
+  }
+  if (bpt != 4) return nullptr;
+  switch (tpr) {
+    case 64: return (const void*)row_fwd_kernel<MODE, 4, 64, SR, HG>;
+    case 128: return (const void*)row_fwd_kernel<MODE, 4, 128, SR, HG>;
+    case 256: return (const void*)row_fwd_kernel<MODE, 4, 256, SR, HG>;
+    default: return nullptr;
   }
 }
 
