@@ -160,6 +160,25 @@ int mxnorm_bwd(const void* x, const void* dy, const void* gamma, const float* G,
 size_t mxnorm_bwd_workspace_size(int64_t T, int64_t D);
 
 /*
+ * Block-scaled MXFP8 GEMM on the tcgen05 tensor cores (MXNorm page, technical
+ * summary section 2.3: MXNormLinear feeds the MX-cast activations into an MX
+ * matmul; "Recipes for Pre-training LLMs with MXFP8": MXFP8-E4M3 operands):
+ *   C[m, n] = sum_k A(m, k) * B(n, k),
+ *   A(m, k) = E4M3(a_q[m, k]) * 2^(scale(m, k/32) - 127), B likewise,
+ * accumulated in fp32, written as bf16.
+ * a_q   uint8 [M, K] E4M3 codes, row-major (K contiguous) -- mxnorm_fwd's q
+ * a_s   uint8 scales of A in the MXN_SCALES_MMA layout (M x K/32 bytes)
+ * b_q   uint8 [N, K] E4M3 codes, K contiguous (the weight transposed) --
+ *       mxfp8_cast of W^T
+ * b_s   uint8 scales of B in the MXN_SCALES_MMA layout (N x K/32 bytes)
+ * c     bf16 [M, N] row-major (written)
+ * Requires M % 128 == 0, N % 256 == 0, K % 128 == 0 (MXN_ERR_UNSUPPORTED
+ * otherwise); M = 0 or N = 0 is a no-op.  One CTA per 128 x 256 tile.
+ */
+int mxfp8_gemm(const void* a_q, const void* a_s, const void* b_q, const void* b_s, void* c, int64_t M,
+               int64_t N, int64_t K, void* stream);
+
+/*
  * mxnorm_bwd without a workspace argument, for callers that cannot allocate
  * device memory when they call: code recorded into a CUDA graph whose memory
  * plan is fixed up front, plugins inside an engine that owns every allocation,

@@ -9,6 +9,7 @@
 #include <tuple>
 
 #include "fwd_dispatch.h"
+#include "gemm_mxfp8.h"
 #include "mxnorm.h"
 #include "row_bwd.cuh"
 #include "row_fwd.cuh"
@@ -582,6 +583,34 @@ int mxnorm_bwd_noalloc(const void* x, const void* dy, const void* gamma, const f
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "dgamma_reduce_kernel launch");
   }
+  return MXN_OK;
+}
+
+int mxfp8_gemm(const void* a_q, const void* a_s, const void* b_q, const void* b_s, void* c, int64_t M,
+               int64_t N, int64_t K, void* stream) {
+  t_err.clear();
+  if (M < 0 || N < 0 || K < 0) return fail(MXN_ERR_ARG, "negative GEMM shape");
+  if (M == 0 || N == 0) return MXN_OK;
+  if (K == 0) return fail(MXN_ERR_UNSUPPORTED, "mxfp8_gemm: K = 0");
+  const void* ptrs[5] = {a_q, a_s, b_q, b_s, c};
+  const char* names[5] = {"a_q", "a_s", "b_q", "b_s", "c"};
+  for (int i = 0; i < 5; ++i) {
+    int rc = check_out(ptrs[i], names[i]);
+    if (rc) return rc;
+  }
+  if (M % gemm_mxfp8_tile_m() || N % gemm_mxfp8_tile_n() || K % gemm_mxfp8_tile_k())
+    return fail(MXN_ERR_UNSUPPORTED, "mxfp8_gemm: M %% %d, N %% %d and K %% %d must be 0 (M=%lld N=%lld K=%lld)",
+                gemm_mxfp8_tile_m(), gemm_mxfp8_tile_n(), gemm_mxfp8_tile_k(), (long long)M, (long long)N,
+                (long long)K);
+  if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return fail(MXN_ERR_UNSUPPORTED, "mxfp8_gemm: shape too large");
+  int rc = injected();
+  if (rc) return rc;
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  const char* why = "";
+  const int e = gemm_mxfp8_launch(a_q, a_s, b_q, b_s, c, (int)M, (int)N, (int)K, dev.status,
+                                  static_cast<cudaStream_t>(stream), &why);
+  if (e) return fail(MXN_ERR_CUDA, "mxfp8_gemm: %s", why);
   return MXN_OK;
 }
 

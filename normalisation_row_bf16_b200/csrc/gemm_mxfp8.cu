@@ -1,0 +1,288 @@
+// gemm_mxfp8.cu -- block-scaled MXFP8 GEMM on the sm_100a tensor cores.
+//
+// The consumer of MXNorm's output (gist.science, "MXNorm: Reusing MXFP block
+// scales for efficient tensor normalisation", technical summary section 2.3:
+// MXNormLinear feeds the MX-cast activations straight into an MX matmul):
+//   C[m, n] = sum_k A(m, k) * B(n, k),  A(m,k) = e4m3(a_q[m,k]) * 2^(a_s[m,k/32] - 127),
+//   B likewise, fp32 accumulation in tensor memory, bf16 output.
+//
+// One CTA computes a 128 x 256 tile of C:
+//  * a producer thread streams 128-element K stages of A (128 x 128 B) and B
+//    (256 x 128 B) into a 4-stage shared-memory ring with TMA tensor copies
+//    (128-byte swizzle, no multicast), and the stage's scale atoms (the
+//    128-row x 4-block, 512-byte tiles of the tcgen05 scale layout) with 1-D
+//    bulk copies;
+//  * an MMA thread copies each stage's scale atoms into tensor memory
+//    (tcgen05.cp 32x128b, replicated to the four lane quarters) and issues four
+//    tcgen05.mma.kind::mxf8f6f4.block_scale (M = 128, N = 256, K = 32 each),
+//    then tcgen05.commit frees the stage when those MMAs retire;
+//  * after the last stage the four warps read the fp32 accumulator out of
+//    tensor memory (tcgen05.ld 32x32b) and write bf16.
+// Every mbarrier wait is bounded; a wait that gives up records itself in the
+// device status word, and the CTA still frees its tensor memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "device_common.cuh"
+#include "gemm_mxfp8.h"
+
+namespace mxn {
+namespace {
+
+constexpr int kTileM = 128, kTileN = 256, kTileK = 128;  // K elements (= bytes) per stage
+constexpr int kStages = 4;
+constexpr int kThreads = 128;
+constexpr uint32_t kABytes = kTileM * kTileK;    // 16 KiB
+constexpr uint32_t kBBytes = kTileN * kTileK;    // 32 KiB
+constexpr uint32_t kSfaBytes = 512;              // one 128 x 4 scale atom
+constexpr uint32_t kSfbBytes = 1024;             // two atoms (256 rows)
+constexpr uint32_t kStageTx = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCol = 0;                  // accumulator: columns 0..255
+constexpr uint32_t kSfCol0 = 256;                // scales: 12 columns per stage
+
+struct Smem {
+  uint8_t a[kStages][kABytes];                   // 1024-aligned (128B swizzle atoms)
+  uint8_t b[kStages][kBBytes];
+  uint8_t sfa[kStages][kSfaBytes];
+  uint8_t sfb[kStages][kSfbBytes];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full;
+  uint32_t tmem_base;
+  uint32_t failed;
+};
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s_plain(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05): start >> 4 in bits 0..13,
+// leading byte offset >> 4 in 16..29, stride byte offset >> 4 in 32..45,
+// version 1 in 46..47, layout type in 61..63 (2 = 128-byte swizzle, 0 = none).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with E8M0 block scales:
+// A, B E4M3 (format 0), both K-major, N >> 3 in bits 17..22, scale format
+// E8M0 in bit 23, M >> 4 in bits 24..28; scale-factor byte ids in 4..5 (B)
+// and 29..30 (A); dense, K = 32.
+__device__ __forceinline__ uint32_t instr_desc(uint32_t sf_id) {
+  return (sf_id << 4) | ((uint32_t)(kTileN >> 3) << 17) | (1u << 23) | ((uint32_t)(kTileM >> 4) << 24) |
+         (sf_id << 29);
+}
+
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_cp_sf(uint32_t tmem, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem), "l"(src_desc) : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 accumulator columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                      const uint8_t* __restrict__ a_s, const uint8_t* __restrict__ b_s,
+                      uint16_t* __restrict__ c, int M, int N, int K, unsigned* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  Smem& S = *reinterpret_cast<Smem*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = blockIdx.x, nt = blockIdx.y;   // tile coordinates
+  const int n_k = K / kTileK;
+  const int kp4 = K / 32;                       // scale columns (K % 128 == 0, so already a multiple of 4)
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    mbar_init(&S.acc_full, 1);
+    S.failed = 0;
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  int n_issued = 0;                             // producer: stages issued
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------- producer
+    for (int kb = 0; kb < n_k; ++kb) {
+      const int s = kb % kStages;
+      const uint32_t ph = (uint32_t)((kb / kStages) & 1);
+      if (!mbar_wait_bounded(&S.empty[s], ph ^ 1u, status)) { atomicOr(&S.failed, 1u); break; }
+      mbar_arrive_expect_tx(&S.full[s], kStageTx);
+      tma_load_2d(S.a[s], &map_a, kb * kTileK, mt * kTileM, &S.full[s]);
+      tma_load_2d(S.b[s], &map_b, kb * kTileK, nt * kTileN, &S.full[s]);
+      // scale atoms: (row tile, 4-block group) -> 512 contiguous bytes
+      bulk_g2s_plain(S.sfa[s], a_s + ((size_t)mt * (kp4 / 4) + kb) * 512, kSfaBytes, &S.full[s]);
+      bulk_g2s_plain(S.sfb[s], b_s + ((size_t)(2 * nt) * (kp4 / 4) + kb) * 512, 512, &S.full[s]);
+      bulk_g2s_plain(S.sfb[s] + 512, b_s + ((size_t)(2 * nt + 1) * (kp4 / 4) + kb) * 512, 512, &S.full[s]);
+      n_issued = kb + 1;
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------- MMA
+    bool ok = true;
+    for (int kb = 0; kb < n_k && ok; ++kb) {
+      const int s = kb % kStages;
+      const uint32_t ph = (uint32_t)((kb / kStages) & 1);
+      if (!mbar_wait_bounded(&S.full[s], ph, status)) { atomicOr(&S.failed, 1u); ok = false; break; }
+      tc_fence_after();
+      const uint32_t sfa_col = kSfCol0 + (uint32_t)s * 12u, sfb_col = sfa_col + 4u;
+      // scale atoms -> tensor memory: 32 rows x 16 B each, 8-row core matrices 128 B apart
+      tmem_cp_sf(tmem + sfa_col, smem_desc(smem_u32(S.sfa[s]), 0, 128, 0));
+      tmem_cp_sf(tmem + sfb_col, smem_desc(smem_u32(S.sfb[s]), 0, 128, 0));
+      tmem_cp_sf(tmem + sfb_col + 4u, smem_desc(smem_u32(S.sfb[s] + 512), 0, 128, 0));
+      const uint32_t a0 = smem_u32(S.a[s]), b0 = smem_u32(S.b[s]);
+#pragma unroll
+      for (int k = 0; k < kTileK / 32; ++k) {
+        // 32 bytes further along the 128-byte swizzled rows; 8-row atoms 1024 B apart
+        const uint64_t ad = smem_desc(a0 + 32u * k, 16, 1024, 2);
+        const uint64_t bd = smem_desc(b0 + 32u * k, 16, 1024, 2);
+        mma_mxf8(tmem + kAccCol, ad, bd, instr_desc((uint32_t)k),
+                 (tmem + sfa_col) | ((uint32_t)k << 30), (tmem + sfb_col) | ((uint32_t)k << 30),
+                 (kb > 0 || k > 0) ? 1u : 0u);
+      }
+      tc_commit(&S.empty[s]);                    // stage free once these MMAs retire
+    }
+    tc_commit(&S.acc_full);                       // accumulator complete (or the loop gave up)
+  }
+
+  // ------------------------------------------------------------ epilogue
+  __syncwarp();
+  const bool got = mbar_wait_bounded(&S.acc_full, 0, status);
+  tc_fence_after();
+  __syncthreads();
+  if (got && S.failed == 0) {
+    const int row = mt * kTileM + warp * 32 + lane;          // this thread's accumulator lane
+    uint16_t* crow = c + (size_t)row * N + (size_t)nt * kTileN;
+#pragma unroll 1
+    for (int cc = 0; cc < kTileN; cc += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + kAccCol + (uint32_t)cc + ((uint32_t)(warp * 32) << 16), r);
+      uint32_t o[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+        o[i] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        *reinterpret_cast<uint4*>(crow + cc + 8 * v) = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  // After a wait gave up, leave no copy in flight: the producer waits (bounded)
+  // for the last issued phase of every stage.
+  if (warp == 0 && lane == 0 && S.failed != 0)
+    for (int j = (n_issued > kStages ? n_issued - kStages : 0); j < n_issued; ++j)
+      mbar_wait_bounded(&S.full[j % kStages], (uint32_t)((j / kStages) & 1), status);
+  __syncwarp();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major uint8 [rows, cols] matrix, boxes of box_rows x 128 bytes, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols};
+  const cuuint32_t box[2] = {(cuuint32_t)kTileK, (cuuint32_t)box_rows};
+  const cuuint32_t elem[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t gemm_mxfp8_smem_bytes() { return sizeof(Smem) + 1024; }
+
+// Launch: returns 0, or -1 (tensor map could not be encoded) / cuda error code.
+int gemm_mxfp8_launch(const void* a_q, const void* a_s, const void* b_q, const void* b_s, void* c, int M,
+                      int N, int K, unsigned* status, cudaStream_t stream, const char** why) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, a_q, M, K, kTileM) || !make_map(&mb, b_q, N, K, kTileN)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return -1;
+  }
+  const size_t smem = sizeof(Smem);
+  cudaError_t e = cudaFuncSetAttribute(gemm_mxfp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) { *why = cudaGetErrorString(e); return (int)e; }
+  dim3 grid(M / kTileM, N / kTileN);
+  gemm_mxfp8_kernel<<<grid, kThreads, smem, stream>>>(ma, mb, static_cast<const uint8_t*>(a_s),
+                                                      static_cast<const uint8_t*>(b_s),
+                                                      static_cast<uint16_t*>(c), M, N, K, status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) { *why = cudaGetErrorString(e); return (int)e; }
+  return 0;
+}
+
+int gemm_mxfp8_tile_m() { return kTileM; }
+int gemm_mxfp8_tile_n() { return kTileN; }
+int gemm_mxfp8_tile_k() { return kTileK; }
+
+}  // namespace mxn

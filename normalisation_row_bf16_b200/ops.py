@@ -31,6 +31,7 @@ SIGNATURES = {
     "mxnorm_bwd": (_I32, [_P, _P, _P, _P, _P, _P, _I64, _I64, _P, _SZ, _P]),
     "mxnorm_bwd_workspace_size": (_SZ, [_I64, _I64]),
     "mxnorm_bwd_noalloc": (_I32, [_P, _P, _P, _P, _P, _P, _I64, _I64, _P]),
+    "mxfp8_gemm": (_I32, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "mxnorm_last_error": (ctypes.c_char_p, []),
     "mxnorm_device_status": (_I32, [_P]),
     "mxnorm_set_tuning": (_I32, [_I32, _I32, _I32]),
@@ -197,6 +198,19 @@ def mxnorm_bwd_noalloc(x, dy, gamma, G, dx=None, dgamma=None, want_dgamma: bool 
     _check(lib().mxnorm_bwd_noalloc(_ptr(x), _ptr(dy), _ptr(gamma), _ptr(G), _ptr(dx), _ptr(dgamma),
                                     T, D, _stream(stream)))
     return dx, dgamma
+
+
+def mxfp8_gemm(a_q, a_s, b_q, b_s, M: int, N: int, K: int, c=None, stream=None):
+    """C bf16 [M, N] = dequant(A) @ dequant(B)^T; scales in the MMA layout."""
+    for t in (a_q, a_s, b_q, b_s):
+        if not t.is_cuda or t.dtype != torch.uint8:
+            raise ValueError("GEMM operands must be uint8 CUDA tensors")
+    if a_q.numel() != M * K or b_q.numel() != N * K:
+        raise ValueError("code tensors do not match M, N, K")
+    if c is None:
+        c = torch.empty(M, N, dtype=torch.bfloat16, device=a_q.device)
+    _check(lib().mxfp8_gemm(_ptr(a_q), _ptr(a_s), _ptr(b_q), _ptr(b_s), _ptr(c), M, N, K, _stream(stream)))
+    return c
 
 
 def device_status(stream=None) -> int:

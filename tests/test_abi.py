@@ -129,3 +129,17 @@ def test_python_binding_refuses_cpu_tensors(L):
     x = torch.zeros(4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ops.mxnorm_fwd(x)
+
+
+def test_gemm_argument_checks(L):
+    f = L.mxfp8_gemm
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 256, 128, None) == ops.MXN_OK        # empty
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, -1, 256, 128, None) == ops.MXN_ERR_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 0, None) == ops.MXN_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 100, 256, 128, None) == ops.MXN_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 200, 128, None) == ops.MXN_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 96, None) == ops.MXN_ERR_UNSUPPORTED
+    assert f(None, FAKE, FAKE, FAKE, FAKE, 128, 256, 128, None) == ops.MXN_ERR_ARG
+    assert f(FAKE, FAKE, MISALIGNED, FAKE, FAKE, 128, 256, 128, None) == ops.MXN_ERR_ARG
+    L.mxnorm_debug_fail_next(1)
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 128, None) == ops.MXN_ERR_CUDA
