@@ -592,6 +592,7 @@ int mxfp8_gemm(const void* a_q, const void* a_s, const void* b_q, const void* b_
   if (M < 0 || N < 0 || K < 0) return fail(MXN_ERR_ARG, "negative GEMM shape");
   if (M == 0 || N == 0) return MXN_OK;
   if (K == 0) return fail(MXN_ERR_UNSUPPORTED, "mxfp8_gemm: K = 0");
+  t_empty = false;  // every operand pointer is required from here on
   const void* ptrs[5] = {a_q, a_s, b_q, b_s, c};
   const char* names[5] = {"a_q", "a_s", "b_q", "b_s", "c"};
   for (int i = 0; i < 5; ++i) {
