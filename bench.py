@@ -354,6 +354,11 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
                   "d2h_bytes_per_step": T * D + T * (D // 32) + 4 * T,
                   "steps": Ke, "ms_per_step": round(te_ms, 4)}
 
+    # Downstream block-scaled MXFP8 GEMM (MXNormLinear): the MXNorm output of
+    # an 8192 x 4096 N(0,1) batch times the fused QKV weight [4096 x 6144].
+    if D == 4096 and T % 128 == 0:
+        out["gemm"] = run_gemm_leg(args, w, rank, world, dev, barrier)
+
     # CPU oracle on the host cores: rank 0, one GPU only
     if rank == 0 and world == 1:
         import oracle
@@ -367,6 +372,50 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
                                "cores": oracle.num_threads(), "kind": "oracle",
                                "sample": f"all {T} rows of the workload, once ({dt:.2f} s)"}
     return out
+
+
+def run_gemm_leg(args, w, rank, world, dev, barrier):
+    import torch
+    import torch.distributed as dist
+    from normalisation_row_bf16_b200 import ops, synthetic
+
+    T, K, N = w["T"], w["D"], 6144
+    x = synthetic.activations(T, K, "normal", seed=rank, device=dev)
+    g = synthetic.gamma(K, seed=rank, device=dev)
+    wt = synthetic.gemm_weight(N, K, seed=rank, device=dev)
+    aq, a_s, _ = ops.mxnorm_fwd(x, g, 2.0, scale_layout=ops.SCALES_MMA)
+    bq, b_s = ops.mxfp8_cast(wt, scale_layout=ops.SCALES_MMA)
+    c = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
+    for _ in range(max(3, args.warmup)):
+        ops.mxfp8_gemm(aq, a_s, bq, b_s, T, N, K, c=c)
+    Kg = max(1, min(args.steps, 200))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(Kg):
+            ops.mxfp8_gemm(aq, a_s, bq, b_s, T, N, K, c=c)
+    graph.replay()
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    graph.replay()
+    t1.record()
+    barrier()
+    del graph
+    ms = t0.elapsed_time(t1) / Kg
+    tm = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+    ms = float(tm[0])
+    flops = 2.0 * T * N * K
+    peaks, src = measured_peaks()
+    bf16 = float(peaks.get("bf16_tflops", 1590.0))
+    fp8_peak = 2.0 * bf16        # nominal dense fp8 : bf16 ratio is 2 (4.5 vs 2.25 PFLOP/s)
+    tflops = world * flops / (ms * 1e-3) / 1e12
+    return {"shape_MNK": [T, N, K], "ms": round(ms, 5), "steps": Kg, "TFLOPs": round(tflops, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tflops / world, 1), "peak": round(fp8_peak, 1),
+                         "unit": "TFLOP/s", "frac": round(tflops / world / fp8_peak, 4),
+                         "peak_source": f"{src} bf16 x 2 (nominal fp8/bf16 ratio)"},
+            "kernel": "gemm_mxfp8_kernel (tcgen05 mxf8f6f4 block_scale, 128x256 tiles)"}
 
 
 # ---------------------------------------------------------- reference arm

@@ -231,6 +231,15 @@ int mxnorm_set_tuning(int consumer_threads, int stages, int ctas_per_sm);
  */
 void mxnorm_debug_fail_next(int count);
 
+/*
+ * Test hook for the bounded waits: launches one thread that waits on an
+ * mbarrier nothing ever arrives on, for at most limit_ns (0 < limit_ns <= 2 s).
+ * The wait gives up, sets the device status word (mxnorm_device_status then
+ * returns MXN_ERR_TIMEOUT) and writes 1 to the device int *gave_up; the
+ * context stays usable.  No trap, no fault.
+ */
+int mxnorm_debug_wait_timeout(uint64_t limit_ns, int* gave_up, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -386,6 +386,18 @@ int noalloc_scratch(float** out) {
   return MXN_OK;
 }
 
+// Test kernel for the bounded-wait mechanism: one thread initialises an
+// mbarrier that expects one arrival, never arrives, and waits on it for at most
+// limit_ns; the wait gives up, records itself in the status word and returns.
+__global__ void wait_timeout_probe_kernel(uint64_t limit_ns, unsigned* status, int* gave_up) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    *gave_up = mbar_wait_limit(&bar, 0, limit_ns, status) ? 0 : 1;
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -612,6 +624,20 @@ int mxfp8_gemm(const void* a_q, const void* a_s, const void* b_q, const void* b_
   const int e = gemm_mxfp8_launch(a_q, a_s, b_q, b_s, c, (int)M, (int)N, (int)K, dev.status,
                                   static_cast<cudaStream_t>(stream), &why);
   if (e) return fail(MXN_ERR_CUDA, "mxfp8_gemm: %s", why);
+  return MXN_OK;
+}
+
+int mxnorm_debug_wait_timeout(uint64_t limit_ns, int* gave_up, void* stream) {
+  t_err.clear();
+  t_empty = false;
+  int rc = check_out(gave_up, "gave_up");
+  if (rc) return rc;
+  if (limit_ns == 0 || limit_ns > 2000000000ull) return fail(MXN_ERR_ARG, "limit_ns = %llu", (unsigned long long)limit_ns);
+  DeviceInfo dev;
+  if ((rc = device_info(&dev))) return rc;
+  wait_timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, dev.status, gave_up);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "wait_timeout_probe_kernel launch");
   return MXN_OK;
 }
 

@@ -77,6 +77,20 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
+// As mbar_wait_bounded below, with an explicit limit.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                                unsigned* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
+    if (global_timer_ns() - t0 > limit_ns) {
+      atomicOr(status, kStatusWaitTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
 // Wait until the phase of `bar` with the given parity has completed, for at
 // most kWaitLimitNs.  Returns false (and records the timeout in *status) if
 // the wait gave up.  Sleeping waits: the clock is read once per ~20 us wake-up.

@@ -36,6 +36,7 @@ SIGNATURES = {
     "mxnorm_device_status": (_I32, [_P]),
     "mxnorm_set_tuning": (_I32, [_I32, _I32, _I32]),
     "mxnorm_debug_fail_next": (None, [_I32]),
+    "mxnorm_debug_wait_timeout": (_I32, [_U64, _P, _P]),
 }
 
 _lib = None
