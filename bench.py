@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--workload", default="llama8b_8192x4096_outliers_p2")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the two-pass comparator, e2e and CPU baseline legs")
+    ap.add_argument("--sweep", action="store_true",
+                    help="also time MXNorm forward over the sweep shapes (16384 x {2048..16384}, p in {1,2,4,inf}, RNE/SR)")
     ap.add_argument("--soak-s", type=float, default=0.5,
                     help="untimed back-to-back steps before timing, so clocks settle under load")
     return ap.parse_args()
@@ -354,10 +356,26 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
                   "d2h_bytes_per_step": T * D + T * (D // 32) + 4 * T,
                   "steps": Ke, "ms_per_step": round(te_ms, 4)}
 
+    # Stochastic-rounding forward and the backward on the same batch.
+    out["sr_fwd"] = run_graph_leg(args, world, dev, barrier,
+                                  lambda i: ops.mxnorm_fwd(xs[i % n_sets], g, p, rounding=ops.SR, seed=i),
+                                  algorithmic_bytes(T, D), "row_fwd_kernel<MXNorm, SR>")
+    dy = synthetic_grad(T, D, dev)
+    dxb = torch.empty_like(xs[0])
+    _, _, Gb = ops.mxnorm_fwd(xs[0], g, p)
+    dgb = torch.empty(D, dtype=torch.bfloat16, device=dev)
+    wsb = torch.empty(max(16, ops.bwd_workspace_bytes(T, D)), dtype=torch.uint8, device=dev)
+    out["bwd"] = run_graph_leg(args, world, dev, barrier,
+                               lambda i: ops.mxnorm_bwd(xs[i % n_sets], dy, g, Gb, dx=dxb, dgamma=dgb, workspace=wsb),
+                               bwd_bytes(T, D, wsb.numel()), "row_bwd_kernel + dgamma_reduce_kernel")
+
     # Downstream block-scaled MXFP8 GEMM (MXNormLinear): the MXNorm output of
     # an 8192 x 4096 N(0,1) batch times the fused QKV weight [4096 x 6144].
     if D == 4096 and T % 128 == 0:
         out["gemm"] = run_gemm_leg(args, w, rank, world, dev, barrier)
+
+    if args.sweep:
+        out["sweep"] = run_sweep(args, world, dev, barrier)
 
     # CPU oracle on the host cores: rank 0, one GPU only
     if rank == 0 and world == 1:
@@ -372,6 +390,76 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
                                "cores": oracle.num_threads(), "kind": "oracle",
                                "sample": f"all {T} rows of the workload, once ({dt:.2f} s)"}
     return out
+
+
+def synthetic_grad(T, D, dev):
+    from normalisation_row_bf16_b200 import synthetic
+    return synthetic.upstream_grad(T, D, seed=0, device=dev)
+
+
+def bwd_bytes(T, D, ws_bytes):
+    # read x, dy (2 B/elem each), write dx (2 B/elem); G, gamma; partial sums
+    # written and read once; dgamma written
+    return 6 * T * D + 4 * T + 2 * D + 2 * ws_bytes + 2 * D
+
+
+def run_graph_leg(args, world, dev, barrier, fn, nbytes, kernel):
+    """Time fn(i) for K steps as one replayed CUDA graph; GB/s vs the HBM peak."""
+    import torch
+    import torch.distributed as dist
+    for i in range(max(3, args.warmup)):
+        fn(i)
+    K = max(1, min(args.steps, 500))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(K):
+            fn(i)
+    graph.replay()
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    graph.replay()
+    t1.record()
+    barrier()
+    del graph
+    tm = torch.tensor([t0.elapsed_time(t1) / K], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+    ms = float(tm[0])
+    peaks, src = measured_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms": round(ms, 5), "steps": K, "GBps": round(world * gbs, 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(gbs / peak, 4), "algorithmic_bytes_per_launch": int(nbytes)},
+            "kernel": kernel}
+
+
+def run_sweep(args, world, dev, barrier):
+    import math as _m
+    import torch
+    from normalisation_row_bf16_b200 import ops, synthetic
+    res = []
+    for D in (2048, 4096, 8192, 16384):
+        T = 16384
+        x = synthetic.activations(T, D, "student_t", seed=1, device=dev)
+        n_rot = max(1, math.ceil(3 * L2_BYTES / (T * D * 2)))
+        xs2 = [x] + [x.clone() for _ in range(n_rot - 1)]
+        q = torch.empty(T, D, dtype=torch.uint8, device=dev)
+        sc = torch.empty(T, D // 32, dtype=torch.uint8, device=dev)
+        G = torch.empty(T, dtype=torch.float32, device=dev)
+        for p in (1.0, 2.0, 4.0, _m.inf):
+            for rnd in (ops.RNE, ops.SR):
+                r = run_graph_leg(args, world, dev, barrier,
+                                  lambda i: ops.mxnorm_fwd(xs2[i % len(xs2)], None, p, rounding=rnd, seed=0,
+                                                           q=q, scales=sc, G=G),
+                                  algorithmic_bytes(T, D) - 2 * D, "row_fwd_kernel<MXNorm>")
+                res.append({"T": T, "D": D, "p": "inf" if _m.isinf(p) else p,
+                            "rounding": "sr" if rnd == ops.SR else "rne", "ms": r["ms"],
+                            "GBps": r["GBps"], "frac": r["roofline"]["frac"]})
+        del x, xs2
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_gemm_leg(args, w, rank, world, dev, barrier):
