@@ -5,7 +5,7 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
 code with the CUDA library ``normalisation_row_bf16_b200`` and never imports it.
 
 The arithmetic lives in ``mxnorm_oracle.c`` (plain C, fp64 / long-double
-statistics, exact E4M3 / E8M0 rounding); this module compiles it with gcc on
+statistics, exact E4M3 / E2M1 / E8M0 rounding); this module compiles it with gcc on
 first use and marshals numpy arrays.  Every function names the passage it
 follows in the C source.
 
@@ -55,6 +55,11 @@ def _load():
         lib.oracle_e4m3_rne_many.argtypes = [P, i64, P]
         lib.oracle_e4m3_sr_many.argtypes = [P, P, i64, P]
         lib.oracle_e8m0_exponent_many.argtypes = [P, i64, P]
+        lib.oracle_e2m1_rne_many.argtypes = [P, i64, P]
+        lib.oracle_e2m1_sr_many.argtypes = [P, P, i64, P]
+        lib.oracle_mx_exponent_many.argtypes = [P, i64, f64, P]
+        lib.oracle_e2m1_value.argtypes = [i32]
+        lib.oracle_e2m1_value.restype = f64
         lib.oracle_sr_words.argtypes = [u64, P, i64, P]
         lib.oracle_philox4x32_10.argtypes = [P, P, P]
         lib.oracle_pmean.argtypes = [P, i64, f64]
@@ -63,10 +68,14 @@ def _load():
         lib.oracle_e4m3_value.restype = f64
         lib.oracle_mxnorm_fwd.argtypes = [P, i64, P, i64, P, i64, f64, P, P, P, P, i32, u64, i32]
         lib.oracle_mxfp8_cast.argtypes = [P, i64, i64, P, i64, P, P, i32, u64, i32]
+        lib.oracle_mxnorm_fwd_ex.argtypes = [P, i64, P, i64, P, i64, f64, P, P, P, P, i32, u64,
+                                             i32, i32, i32]
+        lib.oracle_mx_cast_ex.argtypes = [P, i64, P, i64, P, i64, P, P, i32, u64, i32, i32]
         lib.oracle_rmsnorm.argtypes = [P, i64, P, i64, P, i64, f32, P, i32]
         lib.oracle_mxnorm_bwd.argtypes = [P, P, P, P, i64, P, i64, i32, P, P]
         lib.oracle_mxfp8_gemm_entries.argtypes = [P, P, P, P, i64, i64, i64, i64, P, P, P, i32]
         for name in ("oracle_mxnorm_fwd", "oracle_mxfp8_cast", "oracle_rmsnorm",
+                     "oracle_mxnorm_fwd_ex", "oracle_mx_cast_ex",
                      "oracle_mxnorm_bwd", "oracle_mxfp8_gemm_entries"):
             getattr(lib, name).restype = i32
         lib.oracle_num_threads.restype = i32
@@ -138,6 +147,40 @@ def e8m0_exponent(a) -> np.ndarray:
     return out
 
 
+def e2m1_rne(v) -> np.ndarray:
+    """fp32 -> E2M1 4-bit code (sign in bit 3), nearest-even, saturating to 6."""
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float32))
+    out = np.empty(v.shape, np.uint8)
+    _load().oracle_e2m1_rne_many(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def e2m1_sr(v, r32) -> np.ndarray:
+    """fp32 -> E2M1 code by stochastic rounding with the given 32-bit words."""
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float32))
+    r = np.ascontiguousarray(np.asarray(r32, dtype=np.uint32))
+    assert r.shape == v.shape
+    out = np.empty(v.shape, np.uint8)
+    _load().oracle_e2m1_sr_many(_ptr(v), _ptr(r), v.size, _ptr(out))
+    return out
+
+
+def e2m1_value(code: int) -> float:
+    return float(_load().oracle_e2m1_value(int(code)))
+
+
+def mx_exponent(a, elem_max: float) -> np.ndarray:
+    """Smallest e in [-127, 127] with |a| <= elem_max * 2^e (128 for NaN / inf)."""
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    out = np.empty(a.shape, np.int32)
+    _load().oracle_mx_exponent_many(_ptr(a), a.size, float(elem_max), _ptr(out))
+    return out
+
+
+FMT = {"e4m3": 0, "e2m1": 1}
+STAT = {"absmax": 0, "scale_exp": 1}
+
+
 def philox4x32_10(ctr, key) -> np.ndarray:
     c = np.ascontiguousarray(np.asarray(ctr, dtype=np.uint32).reshape(4))
     k = np.ascontiguousarray(np.asarray(key, dtype=np.uint32).reshape(2))
@@ -183,6 +226,44 @@ def mxnorm_fwd(x, gamma=None, p: float = 2.0, rows=None, G_in=None, rounding: in
     if rc != 0:
         raise ValueError("oracle_mxnorm_fwd: bad arguments")
     return q, s, G
+
+
+def mxnorm_fwd_ex(x, gamma=None, p: float = 2.0, rows=None, G_in=None, rounding: int = 0,
+                  seed: int = 0, stat: str = "absmax", fmt: str = "e4m3", nthreads: int = 0):
+    """MXNorm forward with a choice of block statistic ("absmax", or "scale_exp":
+    the block's power-of-two scale) and element format ("e4m3", or "e2m1" with
+    two codes per byte, q uint8 [n, D/2]).  Returns (q, scales, G)."""
+    xu = _u16(x)
+    T, D = xu.shape
+    g = _u16(gamma)
+    r, n = _rows(rows, T)
+    Gi = None if G_in is None else np.ascontiguousarray(np.asarray(G_in, np.float32).reshape(n))
+    q = np.empty((n, D // 2 if fmt == "e2m1" else D), np.uint8)
+    s = np.empty((n, D // 32), np.uint8)
+    G = np.empty(n, np.float32)
+    rc = _load().oracle_mxnorm_fwd_ex(_ptr(xu), D, _ptr(g), n, _ptr(r), D, float(p), _ptr(Gi),
+                                      _ptr(q), _ptr(s), _ptr(G), int(rounding),
+                                      ctypes.c_uint64(seed), STAT[stat], FMT[fmt], int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_mxnorm_fwd_ex: bad arguments")
+    return q, s, G
+
+
+def mx_cast(x, gamma=None, rows=None, rounding: int = 0, seed: int = 0, fmt: str = "e4m3",
+            nthreads: int = 0):
+    """MX quantisation of x, or of fl32(x * gamma) along each row (the folded
+    MXNormLinear weight): (q uint8 [n, D] or [n, D/2], scales uint8 [n, D/32])."""
+    xu = _u16(x)
+    T, D = xu.shape
+    g = _u16(gamma)
+    r, n = _rows(rows, T)
+    q = np.empty((n, D // 2 if fmt == "e2m1" else D), np.uint8)
+    s = np.empty((n, D // 32), np.uint8)
+    rc = _load().oracle_mx_cast_ex(_ptr(xu), D, _ptr(g), n, _ptr(r), D, _ptr(q), _ptr(s),
+                                   int(rounding), ctypes.c_uint64(seed), FMT[fmt], int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_mx_cast_ex: bad arguments")
+    return q, s
 
 
 def mxfp8_cast(x, rows=None, rounding: int = 0, seed: int = 0, nthreads: int = 0):

@@ -29,6 +29,17 @@
  *  [PX]  Philox4x32-10: Salmon, Moraes, Dror, Shaw, "Parallel random numbers:
  *        as easy as 1, 2, 3", SC'11 (multipliers, Weyl key increments, round
  *        function S-box as published there).
+ *  [F4]  The FP4 variant the MXNorm summary reports a layer speedup for
+ *        (section 3, "NVFP4"; the related-papers lists on the same pages train
+ *        in FP4).  The pages do not define the element format; the reading
+ *        adopted is the E2M1 element of the OCP Microscaling (MX) v1.0 format
+ *        (1 sign, 2 exponent bits with bias 1, 1 mantissa bit, no infinity or
+ *        NaN: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) in blocks of 32 with one
+ *        E8M0 scale (MXFP4), the scale rounded up as in [RC] with 6 in place
+ *        of 448.
+ *  [SE]  Scale reuse (the MXNorm title: reusing the block scales): the block
+ *        statistic m_k replaced by the block's own power-of-two scale 2^e_k,
+ *        e_k the [RC] exponent of m_k.
  *
  * Precision: statistics (G, RMS, backward sums) in long double / double.
  * Where floating point decides an integer code, the oracle takes that decision
@@ -47,6 +58,9 @@
 
 #define ORACLE_BLOCK 32          /* MX block size B [MX 2.1] */
 #define E4M3_MAX 448.0           /* [F8] */
+#define E2M1_MAX 6.0             /* [F4] */
+#define ORACLE_FMT_E4M3 0
+#define ORACLE_FMT_E2M1 1
 
 /* ---------------------------------------------------------------- helpers */
 
@@ -149,6 +163,67 @@ uint8_t oracle_e4m3_sr(float v, uint32_t r32)
     return sign | e4m3_encode_grid(r);
 }
 
+/* ------------------------------------------------------------ E2M1 [F4] */
+
+/* Value of a non-negative E2M1 code c in [0, 7]. */
+double oracle_e2m1_value(int c)
+{
+    int ex = (c >> 1) & 3, man = c & 1;
+    if (ex == 0) return 0.5 * man;                   /* subnormal: man * 2^-1 */
+    return ldexp(1.0 + man / 2.0, ex - 1);           /* (1 + man/2) * 2^(ex-1) */
+}
+
+/* Spacing of the E2M1 grid around a magnitude a < 6. */
+static double e2m1_step(double a)
+{
+    if (a < 1.0) return 0.5;          /* below the smallest normal: subnormal step */
+    int E;
+    frexp(a, &E);
+    return ldexp(1.0, (E - 1) - 1);   /* 1 fraction bit in binade [2^(E-1), 2^E) */
+}
+
+/* Code of a non-negative grid value r (0 <= r <= 6). */
+static uint8_t e2m1_encode_grid(double r)
+{
+    if (r < 1.0) return (uint8_t)(r / 0.5);
+    int E;
+    double f = frexp(r, &E);
+    int b = E - 1;
+    int man = (int)((2.0 * f - 1.0) * 2.0);
+    return (uint8_t)(((b + 1) << 1) | man);
+}
+
+/* fp32 -> E2M1 (4-bit code, sign in bit 3), round to nearest, ties to the
+   even code, saturating to +-6.  E2M1 has no NaN: a NaN gives the saturated
+   magnitude with its sign bit (the MX row code never passes one here). */
+uint8_t oracle_e2m1_rne(float v)
+{
+    uint8_t sign = signbit(v) ? 0x8 : 0x0;
+    if (isnan(v)) return sign | 0x7;
+    double a = fabs((double)v);
+    if (a >= E2M1_MAX) return sign | 0x7;
+    double step = e2m1_step(a);
+    double n = a / step;
+    double k = floor(n), rem = n - k;
+    if (rem > 0.5 || (rem == 0.5 && fmod(k, 2.0) == 1.0)) k += 1.0;
+    return sign | e2m1_encode_grid(k * step);
+}
+
+/* fp32 -> E2M1 by stochastic rounding [SR], as oracle_e4m3_sr on the E2M1 grid. */
+uint8_t oracle_e2m1_sr(float v, uint32_t r32)
+{
+    uint8_t sign = signbit(v) ? 0x8 : 0x0;
+    if (isnan(v)) return sign | 0x7;
+    double a = fabs((double)v);
+    if (a >= E2M1_MAX) return sign | 0x7;
+    double step = e2m1_step(a);
+    double lo = floor(a / step) * step;
+    double hi = lo + step;
+    double frac = (a - lo) / (hi - lo);
+    double r = ((double)r32 < frac * 4294967296.0) ? hi : lo;
+    return sign | e2m1_encode_grid(r);
+}
+
 /* ---------------------------------------------------------- E8M0 [RC] */
 
 /* Smallest integer e in [-127, 127] with a <= 448 * 2^e ("scale rounded up so
@@ -158,6 +233,16 @@ int oracle_e8m0_exponent(double a)
     if (!(a <= DBL_MAX)) return 128;
     for (int e = -127; e <= 127; ++e)
         if (a <= ldexp(E4M3_MAX, e)) return e;
+    return 128;
+}
+
+/* The same rule for an element format whose largest magnitude is elem_max
+   [RC][F4]: smallest e in [-127, 127] with a <= elem_max * 2^e. */
+int oracle_mx_exponent(double a, double elem_max)
+{
+    if (!(a <= DBL_MAX)) return 128;
+    for (int e = -127; e <= 127; ++e)
+        if (a <= ldexp(elem_max, e)) return e;
     return 128;
 }
 
@@ -218,15 +303,20 @@ double oracle_pmean(const double *m, int64_t K, double p) { return (double)pmean
 
 /* ------------------------------------------- one row of MX quantisation */
 
-/* Quantise one row y[0..D) (fp32 values) to E4M3 codes + E8M0 scales [RC][F8].
+/* Quantise one row y[0..D) (fp32 values) to MX codes + E8M0 scales [RC].
+   fmt: ORACLE_FMT_E4M3 [F8] (one byte per code) or ORACLE_FMT_E2M1 [F4] (two
+   codes per byte, the even column in the low nibble; D/2 bytes per row).
    rounding: 0 = nearest-even, 1 = stochastic with Philox words.
    A block holding an infinity or a NaN (outside the method's contract) gets
-   the NaN scale 0xFF and the positive NaN code 0x7F for every element: the
-   sign of a NaN made by 0 * inf differs between platforms, so none is kept. */
+   the NaN scale 0xFF and a fixed code for every element (E4M3: the positive
+   NaN 0x7F, the sign of a NaN made by 0 * inf differing between platforms;
+   E2M1, which has no NaN: 0x7). */
 static void mx_quantise_row(const float *y, int64_t D, uint8_t *q, uint8_t *scales,
-                            int rounding, uint64_t seed, uint64_t row)
+                            int rounding, uint64_t seed, uint64_t row, int fmt)
 {
     int64_t K = D / ORACLE_BLOCK;
+    const int fp4 = (fmt == ORACLE_FMT_E2M1);
+    if (fp4) memset(q, 0, (size_t)(D / 2));
     for (int64_t k = 0; k < K; ++k) {
         const float *yb = y + k * ORACLE_BLOCK;
         double a = 0.0;                                   /* block absmax of y */
@@ -236,15 +326,22 @@ static void mx_quantise_row(const float *y, int64_t D, uint8_t *q, uint8_t *scal
             if (!(v <= DBL_MAX)) nonfinite = 1;
             else if (v > a) a = v;
         }
-        int e = nonfinite ? 128 : oracle_e8m0_exponent(a);
+        int e = nonfinite ? 128 : (fp4 ? oracle_mx_exponent(a, E2M1_MAX) : oracle_e8m0_exponent(a));
         scales[k] = e8m0_code(e);
         for (int i = 0; i < ORACLE_BLOCK; ++i) {
             int64_t col = k * ORACLE_BLOCK + i;
-            if (e == 128) { q[col] = 0x7F; continue; }           /* non-finite block: NaN code */
-            float inv_scale = ldexpf(1.0f, -e);           /* 2^-e, exact in fp32 */
-            float v = yb[i] * inv_scale;                  /* fp32 product, as the kernel */
-            if (rounding == 0) q[col] = oracle_e4m3_rne(v);
-            else q[col] = oracle_e4m3_sr(v, sr_word(seed, row * (uint64_t)D + (uint64_t)col));
+            uint8_t c;
+            if (e == 128) {
+                c = fp4 ? 0x7 : 0x7F;                     /* non-finite block */
+            } else {
+                float inv_scale = ldexpf(1.0f, -e);       /* 2^-e, exact in fp32 */
+                float v = yb[i] * inv_scale;              /* fp32 product, as the kernel */
+                uint32_t r32 = rounding ? sr_word(seed, row * (uint64_t)D + (uint64_t)col) : 0u;
+                if (fp4) c = rounding ? oracle_e2m1_sr(v, r32) : oracle_e2m1_rne(v);
+                else c = rounding ? oracle_e4m3_sr(v, r32) : oracle_e4m3_rne(v);
+            }
+            if (fp4) q[col / 2] |= (uint8_t)(c << (4 * (col & 1)));
+            else q[col] = c;
         }
     }
 }
@@ -258,21 +355,26 @@ static int64_t pick_row(const int64_t *row_ids, int64_t i) { return row_ids ? ro
 /*
  * For each selected row r (row_ids[i], or i when row_ids is NULL):
  *   m_k   = max_{i in block k} |x_i|                       (exact)
+ *   stat = 1 [SE]: m_k <- 2^e_k, e_k the E8M0 exponent of m_k for the element
+ *          format (non-finite m_k kept)
  *   G     = p-mean of m_k, in long double, rounded to fp32 -> G_out[i]
  *   if G_in is given, G_in[i] replaces G below (two-stage parity: the codes are
  *   re-derived from the kernel's G bits)
  *   s     = fl32(1/G)   (s = 0 when G = 0)
  *   y_j   = fl32(x_j * s), then y_j = fl32(y_j * gamma_j) when gamma is given
- *   scales/codes of y as in mx_quantise_row.
- * Outputs are compact: q[i*D + j], scales[i*K + k], G_out[i].
+ *   scales/codes of y as in mx_quantise_row (fmt: E4M3 or E2M1).
+ * Outputs are compact: q[i*D + j] (E2M1: q[i*D/2 + j/2]), scales[i*K + k], G_out[i].
  */
-int oracle_mxnorm_fwd(const uint16_t *x, int64_t ld_x, const uint16_t *gamma,
-                      int64_t n_rows, const int64_t *row_ids, int64_t D, double p,
-                      const float *G_in, uint8_t *q, uint8_t *scales, float *G_out,
-                      int rounding, uint64_t seed, int nthreads)
+int oracle_mxnorm_fwd_ex(const uint16_t *x, int64_t ld_x, const uint16_t *gamma,
+                         int64_t n_rows, const int64_t *row_ids, int64_t D, double p,
+                         const float *G_in, uint8_t *q, uint8_t *scales, float *G_out,
+                         int rounding, uint64_t seed, int stat, int fmt, int nthreads)
 {
     if (D <= 0 || D % ORACLE_BLOCK != 0 || !(p > 0.0)) return -1;
+    if (fmt != ORACLE_FMT_E4M3 && fmt != ORACLE_FMT_E2M1) return -1;
     int64_t K = D / ORACLE_BLOCK;
+    const int64_t qrow = (fmt == ORACLE_FMT_E2M1) ? D / 2 : D;
+    const double elem_max = (fmt == ORACLE_FMT_E2M1) ? E2M1_MAX : E4M3_MAX;
 #ifdef _OPENMP
     if (nthreads <= 0) nthreads = omp_get_max_threads();
 #pragma omp parallel for schedule(dynamic, 4) num_threads(nthreads)
@@ -288,6 +390,7 @@ int oracle_mxnorm_fwd(const uint16_t *x, int64_t ld_x, const uint16_t *gamma,
                 double v = fabs((double)bf16_to_f32(xr[k * ORACLE_BLOCK + j]));
                 if (isnan(v) || v > mk) mk = v;   /* a NaN, once seen, stays the max */
             }
+            if (stat == 1 && mk <= DBL_MAX) mk = ldexp(1.0, oracle_mx_exponent(mk, elem_max));
             m[k] = mk;
         }
         float G_ref = (float)pmean(m, K, p);
@@ -298,21 +401,35 @@ int oracle_mxnorm_fwd(const uint16_t *x, int64_t ld_x, const uint16_t *gamma,
             float t = bf16_to_f32(xr[j]) * s;
             y[j] = gamma ? t * bf16_to_f32(gamma[j]) : t;
         }
-        mx_quantise_row(y, D, q + i * D, scales + i * K, rounding, seed, (uint64_t)r);
+        mx_quantise_row(y, D, q + i * qrow, scales + i * K, rounding, seed, (uint64_t)r, fmt);
     }
     (void)nthreads;
     return 0;
 }
 
+int oracle_mxnorm_fwd(const uint16_t *x, int64_t ld_x, const uint16_t *gamma,
+                      int64_t n_rows, const int64_t *row_ids, int64_t D, double p,
+                      const float *G_in, uint8_t *q, uint8_t *scales, float *G_out,
+                      int rounding, uint64_t seed, int nthreads)
+{
+    return oracle_mxnorm_fwd_ex(x, ld_x, gamma, n_rows, row_ids, D, p, G_in, q, scales, G_out,
+                                rounding, seed, 0, ORACLE_FMT_E4M3, nthreads);
+}
+
 /* ------------------------------------------------ MXCast [MX 1.2][RC] */
 
-/* Stand-alone MX quantisation of x (no normalisation): y = x. */
-int oracle_mxfp8_cast(const uint16_t *x, int64_t ld_x, int64_t n_rows, const int64_t *row_ids,
-                      int64_t D, uint8_t *q, uint8_t *scales, int rounding, uint64_t seed,
-                      int nthreads)
+/* Stand-alone MX quantisation of x (no normalisation): y = x, or, with a gain
+   gamma, y = fl32(x_j * gamma_j) -- the folded weight W' of MXNormLinear
+   [MX 2.3] when x is a weight stored one output feature per row and gamma
+   runs along the input features. */
+int oracle_mx_cast_ex(const uint16_t *x, int64_t ld_x, const uint16_t *gamma, int64_t n_rows,
+                      const int64_t *row_ids, int64_t D, uint8_t *q, uint8_t *scales,
+                      int rounding, uint64_t seed, int fmt, int nthreads)
 {
     if (D <= 0 || D % ORACLE_BLOCK != 0) return -1;
+    if (fmt != ORACLE_FMT_E4M3 && fmt != ORACLE_FMT_E2M1) return -1;
     int64_t K = D / ORACLE_BLOCK;
+    const int64_t qrow = (fmt == ORACLE_FMT_E2M1) ? D / 2 : D;
 #ifdef _OPENMP
     if (nthreads <= 0) nthreads = omp_get_max_threads();
 #pragma omp parallel for schedule(dynamic, 4) num_threads(nthreads)
@@ -321,11 +438,22 @@ int oracle_mxfp8_cast(const uint16_t *x, int64_t ld_x, int64_t n_rows, const int
         int64_t r = pick_row(row_ids, i);
         const uint16_t *xr = row_ptr(x, ld_x, r);
         float y[D];
-        for (int64_t j = 0; j < D; ++j) y[j] = bf16_to_f32(xr[j]);
-        mx_quantise_row(y, D, q + i * D, scales + i * K, rounding, seed, (uint64_t)r);
+        for (int64_t j = 0; j < D; ++j) {
+            float t = bf16_to_f32(xr[j]);
+            y[j] = gamma ? t * bf16_to_f32(gamma[j]) : t;
+        }
+        mx_quantise_row(y, D, q + i * qrow, scales + i * K, rounding, seed, (uint64_t)r, fmt);
     }
     (void)nthreads;
     return 0;
+}
+
+int oracle_mxfp8_cast(const uint16_t *x, int64_t ld_x, int64_t n_rows, const int64_t *row_ids,
+                      int64_t D, uint8_t *q, uint8_t *scales, int rounding, uint64_t seed,
+                      int nthreads)
+{
+    return oracle_mx_cast_ex(x, ld_x, NULL, n_rows, row_ids, D, q, scales, rounding, seed,
+                             ORACLE_FMT_E4M3, nthreads);
 }
 
 /* ------------------------------------------------- RMSNorm [MX 1.2, 2.2] */
@@ -458,6 +586,21 @@ void oracle_e4m3_sr_many(const float *v, const uint32_t *r, int64_t n, uint8_t *
 void oracle_e8m0_exponent_many(const float *a, int64_t n, int32_t *out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_e8m0_exponent(fabs((double)a[i]));
+}
+
+void oracle_e2m1_rne_many(const float *v, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e2m1_rne(v[i]);
+}
+
+void oracle_e2m1_sr_many(const float *v, const uint32_t *r, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e2m1_sr(v[i], r[i]);
+}
+
+void oracle_mx_exponent_many(const float *a, int64_t n, double elem_max, int32_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_mx_exponent(fabs((double)a[i]), elem_max);
 }
 
 void oracle_sr_words(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *out)
