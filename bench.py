@@ -281,7 +281,7 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
     """Two-pass comparator, end-to-end through host buffers, CPU oracle."""
     import torch
     import torch.distributed as dist
-    from normalisation_row_bf16_b200 import ops
+    from normalisation_row_bf16_b200 import ops, synthetic
 
     T, D, p = w["T"], w["D"], w["p"]
     out = {}
@@ -357,17 +357,25 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
                   "steps": Ke, "ms_per_step": round(te_ms, 4)}
 
     # Stochastic-rounding forward and the backward on the same batch.
+    # Every leg rotates whole input and output sets (> 3x L2), like the headline.
+    outs = [(torch.empty(T, D, dtype=torch.uint8, device=dev), torch.empty(T, D // 32, dtype=torch.uint8, device=dev),
+             torch.empty(T, dtype=torch.float32, device=dev)) for _ in range(n_sets)]
     out["sr_fwd"] = run_graph_leg(args, world, dev, barrier,
-                                  lambda i: ops.mxnorm_fwd(xs[i % n_sets], g, p, rounding=ops.SR, seed=i),
+                                  lambda i: ops.mxnorm_fwd(xs[i % n_sets], g, p, rounding=ops.SR, seed=i,
+                                                           q=outs[i % n_sets][0], scales=outs[i % n_sets][1],
+                                                           G=outs[i % n_sets][2]),
                                   algorithmic_bytes(T, D), "row_fwd_kernel<MXNorm, SR>")
-    dy = synthetic_grad(T, D, dev)
-    dxb = torch.empty_like(xs[0])
-    _, _, Gb = ops.mxnorm_fwd(xs[0], g, p)
+    del outs
+    dys = [synthetic.upstream_grad(T, D, seed=j, device=dev) for j in range(n_sets)]
+    dxs = [torch.empty_like(xs[0]) for _ in range(n_sets)]
+    Gbs = [ops.mxnorm_fwd(xs[j], g, p)[2] for j in range(n_sets)]
     dgb = torch.empty(D, dtype=torch.bfloat16, device=dev)
     wsb = torch.empty(max(16, ops.bwd_workspace_bytes(T, D)), dtype=torch.uint8, device=dev)
     out["bwd"] = run_graph_leg(args, world, dev, barrier,
-                               lambda i: ops.mxnorm_bwd(xs[i % n_sets], dy, g, Gb, dx=dxb, dgamma=dgb, workspace=wsb),
+                               lambda i: ops.mxnorm_bwd(xs[i % n_sets], dys[i % n_sets], g, Gbs[i % n_sets],
+                                                        dx=dxs[i % n_sets], dgamma=dgb, workspace=wsb),
                                bwd_bytes(T, D, wsb.numel()), "row_bwd_kernel + dgamma_reduce_kernel")
+    del dys, dxs, Gbs
 
     # Downstream block-scaled MXFP8 GEMM (MXNormLinear): the MXNorm output of
     # an 8192 x 4096 N(0,1) batch times the fused QKV weight [4096 x 6144].
@@ -390,11 +398,6 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
                                "cores": oracle.num_threads(), "kind": "oracle",
                                "sample": f"all {T} rows of the workload, once ({dt:.2f} s)"}
     return out
-
-
-def synthetic_grad(T, D, dev):
-    from normalisation_row_bf16_b200 import synthetic
-    return synthetic.upstream_grad(T, D, seed=0, device=dev)
 
 
 def bwd_bytes(T, D, ws_bytes):
@@ -443,21 +446,25 @@ def run_sweep(args, world, dev, barrier):
     for D in (2048, 4096, 8192, 16384):
         T = 16384
         x = synthetic.activations(T, D, "student_t", seed=1, device=dev)
-        n_rot = max(1, math.ceil(3 * L2_BYTES / (T * D * 2)))
+        # Whole input + output sets rotate, at least 3x L2 in all, so neither
+        # the reads nor the code writes of one step are served by L2 in the next.
+        per_set = T * D * 3 + T * (D // 32) + 4 * T
+        n_rot = max(2, math.ceil(3 * L2_BYTES / per_set))
         xs2 = [x] + [x.clone() for _ in range(n_rot - 1)]
-        q = torch.empty(T, D, dtype=torch.uint8, device=dev)
-        sc = torch.empty(T, D // 32, dtype=torch.uint8, device=dev)
-        G = torch.empty(T, dtype=torch.float32, device=dev)
+        qs = [torch.empty(T, D, dtype=torch.uint8, device=dev) for _ in range(n_rot)]
+        scs = [torch.empty(T, D // 32, dtype=torch.uint8, device=dev) for _ in range(n_rot)]
+        Gs = [torch.empty(T, dtype=torch.float32, device=dev) for _ in range(n_rot)]
         for p in (1.0, 2.0, 4.0, _m.inf):
             for rnd in (ops.RNE, ops.SR):
                 r = run_graph_leg(args, world, dev, barrier,
-                                  lambda i: ops.mxnorm_fwd(xs2[i % len(xs2)], None, p, rounding=rnd, seed=0,
-                                                           q=q, scales=sc, G=G),
+                                  lambda i: ops.mxnorm_fwd(xs2[i % n_rot], None, p, rounding=rnd, seed=0,
+                                                           q=qs[i % n_rot], scales=scs[i % n_rot],
+                                                           G=Gs[i % n_rot]),
                                   algorithmic_bytes(T, D) - 2 * D, "row_fwd_kernel<MXNorm>")
                 res.append({"T": T, "D": D, "p": "inf" if _m.isinf(p) else p,
                             "rounding": "sr" if rnd == ops.SR else "rne", "ms": r["ms"],
                             "GBps": r["GBps"], "frac": r["roofline"]["frac"]})
-        del x, xs2
+        del x, xs2, qs, scs, Gs
         torch.cuda.empty_cache()
     return res
 

@@ -59,7 +59,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if failed:
         raise RuntimeError("nvcc failed")
     tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.run([nvcc(), "-shared", "-o", tmp, *objs], check=True)
+    subprocess.run([nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs], check=True)
     os.replace(tmp, LIB)
     for o in objs:
         os.remove(o)

@@ -264,14 +264,23 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int64_t T, int D, int64_t ld_x,
   C.rps = C.gthreads / C.tpr;
   C.row_bytes = 2u * (uint32_t)D;
   C.stage_bytes = (uint32_t)C.rps * C.row_bytes;
-  // Default: as many single-row groups as the CTA holds (up to 24 warps), and
-  // extra stages only while 176 KB of shared memory still covers them all.
+  // Defaults measured on B200 with whole input and output sets rotating
+  // through HBM (T = 8192 and 16384): one stage per group, and 512 threads
+  // per CTA for rows of 33..64 blocks and of more than 256, 384 for 65..256
+  // blocks (12 one-warp rows or 6 two-warp rows in flight per SM).  Rows under
+  // 33 blocks, and stochastic rounding (bound by the Philox arithmetic, so it
+  // wants every warp the registers allow), keep the largest CTA with extra
+  // stages while 176 KB covers them.
+  const bool widest = bpt == 1 || sr;
+  const int def_threads = widest ? fwd_max_threads(bpt) : (bpt == 2 || C.tpr > 64 ? 512 : 384);
   if (g_tuning.stages) {
     C.stages = g_tuning.stages;
-  } else {
+  } else if (widest) {
     const int gmax = fwd_max_threads(bpt) / (C.tpr < 32 ? 32 : C.tpr);
     int st = (int)((176u * 1024u) / ((size_t)gmax * C.rps * 2u * (uint32_t)D));
     C.stages = st < 1 ? 1 : (st > 3 ? 3 : st);
+  } else {
+    C.stages = 1;
   }
   // gamma in shared memory: fp32 for up to 64 threads per row (D <= 8192), else bf16
   C.gamma_bytes = gamma_smem ? (uint32_t)align_up((gamma_fp32(C.tpr) ? 4u : 2u) * (uint32_t)D, 128) : 0u;
@@ -284,7 +293,7 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int64_t T, int D, int64_t ld_x,
   if (g_tuning.consumer_threads) {
     ng = g_tuning.consumer_threads / C.gthreads;
   } else {
-    ng = fwd_max_threads(bpt) / C.gthreads;
+    ng = def_threads / C.gthreads;
   }
   int ng_max = fwd_max_threads(bpt) / C.gthreads;
   const size_t fixed = C.gamma_bytes + 16;
@@ -313,7 +322,11 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int64_t T, int D, int64_t ld_x,
   const int64_t max_ctas = (int64_t)sms * occ;
   const int64_t need_ctas = (C.n_row_blocks + ng - 1) / ng;
   const int64_t ctas = need_ctas < max_ctas ? need_ctas : max_ctas;
-  C.ngt = ctas * ng;
+  // Every active group gets R or R - 1 row blocks with R = ceil(blocks / groups):
+  // only as many groups as R rounds need take rows, so no round runs on a
+  // fraction of the groups while the rest idle.
+  const int64_t R = (C.n_row_blocks + ctas * ng - 1) / (ctas * ng);
+  C.ngt = R > 0 ? (C.n_row_blocks + R - 1) / R : 0;
   P->grid = (int)ctas;
   return MXN_OK;
 }

@@ -49,7 +49,7 @@ struct FwdCfg {
   int64_t T;             // rows
   int64_t ld_x;          // row stride of x, elements
   int64_t n_row_blocks;  // ceil(T / rps)
-  int64_t ngt;           // row groups in the grid
+  int64_t ngt;           // row groups that get rows (<= groups in the grid)
   int D, K;              // row length, MX blocks per row
   int tpr, log2_tpr;     // threads per row (power of two)
   int rps;               // rows per row group and stage (> 1 only when tpr < 32)
@@ -317,12 +317,24 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
   constexpr bool has_gamma = (MODE != kModeCast) && HG;
   constexpr bool kGF32 = gamma_fp32(TPR);
 
+  // Global row group, numbered group-major so that the groups of one row
+  // window are spread over all SMs.  Groups at or past C.ngt have no rows (the
+  // planner gives every active group the same number of row blocks, up to one).
+  const int64_t gg = (int64_t)g * gridDim.x + blockIdx.x;
+  const int64_t rb_end = gg < C.ngt ? C.n_row_blocks : 0;
+  const uint64_t pol = policy_evict_first();
+  // The first row copies go out before anything else, so their DRAM latency
+  // overlaps the gamma set-up below.
   if (issuer) {
     for (int s = 0; s < C.stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], n_gwarps);
     }
     fence_barrier_init();
+    for (int s = 0; s < C.stages; ++s) {
+      const int64_t rb = gg + (int64_t)s * C.ngt;
+      if (rb < rb_end) issue_row_block(A.x, C, rb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
+    }
   }
   // gamma -> shared memory in slot order, so that a warp's 16-byte reads of
   // slot j fall on consecutive words: as fp32, half h of slot j of block k
@@ -344,17 +356,6 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
   }
   __syncthreads();
 
-  // Global row group, numbered group-major so that the groups that get one
-  // more row block than the others are spread over all SMs.
-  const int64_t gg = (int64_t)g * gridDim.x + blockIdx.x;
-  const uint64_t pol = policy_evict_first();
-  if (issuer) {
-    for (int s = 0; s < C.stages; ++s) {
-      const int64_t rb = gg + (int64_t)s * C.ngt;
-      if (rb < C.n_row_blocks) issue_row_block(A.x, C, rb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
-    }
-  }
-
   // A wait that gives up marks the kernel failed; threads then keep going
   // without waiting so every named barrier still completes (outputs garbage,
   // accesses in bounds).
@@ -363,7 +364,7 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
   const int bar_id = 1 + g;
   const int rot = (tg >> 1) & 3;           // the same for every block of the thread
   int64_t it = 0;
-  for (int64_t rb = gg; rb < C.n_row_blocks; rb += C.ngt, ++it, par ^= 1) {
+  for (int64_t rb = gg; rb < rb_end; rb += C.ngt, ++it, par ^= 1) {
     const int s = (int)(it % C.stages);
     const uint32_t ph = (uint32_t)((it / C.stages) & 1);
     if (ok) ok = mbar_wait_bounded(&full[s], ph, A.status);
