@@ -87,6 +87,34 @@ enum mxn_scale_layout {
    arguments are invalid. */
 size_t mxnorm_scales_bytes(int64_t T, int64_t D, int layout);
 
+/* Element format of the MX codes. */
+enum mxn_elem_format {
+    MXN_ELEM_E4M3 = 0,  /* MXFP8: one E4M3 code per byte, codes [T, D] */
+    /* MXFP4: E2M1 elements (the FP4 variant the MXNorm summary reports a
+       layer speedup for, section 3; element format as in the OCP
+       Microscaling v1.0 format, which the pages do not spell out): sign,
+       2 exponent bits (bias 1), 1 mantissa bit, magnitudes 0, 0.5, 1, 1.5,
+       2, 3, 4, 6, no infinity or NaN.  Two codes per byte, the even column
+       in bits 0..3: codes [T, D / 2].  Scale rule as for E4M3 with 6 in
+       place of 448; nearest-even saturates to +-6; a block holding NaN or
+       infinity gets scale 0xFF and element code 0x7. */
+    MXN_ELEM_E2M1 = 1
+};
+
+/* Block statistic of the MXNorm p-mean. */
+enum mxn_statistic {
+    MXN_STAT_ABSMAX = 0,     /* m_k = block absmax of x (section 2.1) */
+    /* Scale reuse (the MXNorm title: reusing the MX block scales): m_k is
+       replaced by 2^e_k, e_k the scale exponent of block k of x by the rule
+       above for the element format (a zero block gives 2^-127); infinities
+       and NaN pass through. */
+    MXN_STAT_SCALE_EXP = 1
+};
+
+/* Bytes the codes of a [T, D] tensor occupy in the given element format; 0 if
+   the arguments are invalid. */
+size_t mxnorm_codes_bytes(int64_t T, int64_t D, int elem_format);
+
 /*
  * MXNorm forward (MXNorm page, technical summary section 2.1; gain as in
  * section 2.3).  For every row r of x:
@@ -111,12 +139,45 @@ int mxnorm_fwd(const void* x, const void* gamma, void* q, void* scales, float* G
                int scale_layout, void* stream);
 
 /*
+ * mxnorm_fwd with a choice of element format (enum mxn_elem_format; q holds
+ * mxnorm_codes_bytes(T, D, elem_format) bytes) and of block statistic (enum
+ * mxn_statistic).  Every other argument as in mxnorm_fwd; with MXN_ELEM_E4M3
+ * and MXN_STAT_ABSMAX it is mxnorm_fwd.  Stochastic rounding draws its words
+ * as for E4M3 and rounds between neighbouring E2M1 values.
+ */
+int mxnorm_fwd_ex(const void* x, const void* gamma, void* q, void* scales, float* G_out,
+                  int64_t T, int64_t D, int64_t ld_x, float p, int rounding, uint64_t seed,
+                  int scale_layout, int elem_format, int statistic, void* stream);
+
+/*
  * MX quantisation of x itself (MXCast; MXNorm page, technical summary section
  * 1.2): y = x, then the per-block scale and code of mxnorm_fwd.
  * Same argument meanings as mxnorm_fwd.
  */
 int mxfp8_cast(const void* x, void* q, void* scales, int64_t T, int64_t D, int64_t ld_x,
                int rounding, uint64_t seed, int scale_layout, void* stream);
+
+/*
+ * MXCast with an optional gain along each row and a choice of element format:
+ * y_j = fl32(x_j * gain_j) (exact: a bf16 product fits fp32), or y = x when
+ * gain is NULL; then scales and codes as in mxnorm_fwd_ex.  gain bf16 [D].
+ */
+int mx_cast_ex(const void* x, const void* gain, void* q, void* scales, int64_t T, int64_t D,
+               int64_t ld_x, int rounding, uint64_t seed, int scale_layout, int elem_format,
+               void* stream);
+
+/*
+ * MXNormLinear weight folding (MXNorm page, technical summary section 2.3: the
+ * gain gamma moves into the next layer's weight, W' = diag(gamma) W, and
+ * MXNorm then runs with gamma = NULL).  w is that weight stored the way
+ * mxfp8_gemm reads its B operand: one output feature per row, bf16 [N, ld_w],
+ * K = input features contiguous.  Writes the MX codes and scales of
+ * w[n, k] * gamma[k] (nearest-even): q mxnorm_codes_bytes(N, K, elem_format)
+ * bytes, scales in scale_layout.  gamma bf16 [K], required.  Same as
+ * mx_cast_ex(w, gamma, ..., MXN_ROUND_RNE, 0, ...).
+ */
+int mxnorm_fold_weight(const void* w, const void* gamma, void* q, void* scales, int64_t N,
+                       int64_t K, int64_t ld_w, int elem_format, int scale_layout, void* stream);
 
 /*
  * RMSNorm (MXNorm page, sections 1.1-1.2, the layer MXNorm replaces):

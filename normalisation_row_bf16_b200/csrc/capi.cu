@@ -223,11 +223,20 @@ int check_opt(const void* p, const char* name) {
   return MXN_OK;
 }
 
-const void* fwd_kernel(int mode, bool sr, bool has_gamma, int bpt, int tpr) {
+const void* fwd_kernel(int mode, bool sr, bool has_gamma, int elem, int bpt, int tpr) {
+  if (elem == kElemE2M1) {
+    switch (mode) {
+      case kModeMXNorm:
+        return sr ? fwd_kernel_mxnorm_fp4_sr(bpt, tpr, has_gamma) : fwd_kernel_mxnorm_fp4_rne(bpt, tpr, has_gamma);
+      case kModeCast: return fwd_kernel_cast_fp4(bpt, tpr, sr, has_gamma);
+      default: return nullptr;
+    }
+  }
   switch (mode) {
     case kModeMXNorm:
       return sr ? fwd_kernel_mxnorm_sr(bpt, tpr, has_gamma) : fwd_kernel_mxnorm_rne(bpt, tpr, has_gamma);
-    case kModeCast: return fwd_kernel_cast(bpt, tpr, sr);
+    case kModeCast:
+      return sr ? fwd_kernel_cast_sr(bpt, tpr, has_gamma) : fwd_kernel_cast_rne(bpt, tpr, has_gamma);
     case kModeRMSNorm: return fwd_kernel_rmsnorm(bpt, tpr, has_gamma);
     default: return nullptr;
   }
@@ -244,7 +253,8 @@ struct FwdPlan {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-int plan_fwd(int mode, bool sr, bool gamma_smem, int64_t T, int D, int64_t ld_x, int sms, FwdPlan* P) {
+int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int64_t ld_x, int sms,
+             FwdPlan* P) {
   FwdCfg& C = P->C;
   C = FwdCfg{};
   C.T = T;
@@ -311,7 +321,7 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int64_t T, int D, int64_t ld_x,
   C.red_off = C.bar_off + (uint32_t)(ng * 2 * C.stages * sizeof(uint64_t));
   P->smem = C.red_off + (size_t)ng * 2 * kRedSlots * sizeof(float2);
   P->threads = ng * C.gthreads;
-  P->kernel = fwd_kernel(mode, sr, gamma_smem, bpt, C.tpr);
+  P->kernel = fwd_kernel(mode, sr, gamma_smem, elem, bpt, C.tpr);
   if (!P->kernel) return fail(MXN_ERR_UNSUPPORTED, "no kernel for D = %d", D);
   int occ = 0;
   int rc = occupancy(P->kernel, P->threads, P->smem, &occ);
@@ -347,7 +357,7 @@ int launch_fwd(int mode, bool sr, const FwdArgs& A, int64_t T, int D, int64_t ld
   int rc = device_info(&dev);
   if (rc) return rc;
   FwdPlan P;
-  rc = plan_fwd(mode, sr, A.gamma != nullptr && mode != kModeCast, T, D, ld_x, dev.sms, &P);
+  rc = plan_fwd(mode, sr, A.gamma != nullptr, A.elem, T, D, ld_x, dev.sms, &P);
   if (rc) return rc;
   FwdArgs a = A;
   a.status = dev.status;
@@ -425,7 +435,7 @@ size_t mxnorm_scales_bytes(int64_t T, int64_t D, int layout) {
 
 static int fwd_like(int mode, const void* x, const void* gamma, void* q, void* scales, float* G_out,
                     int64_t T, int64_t D, int64_t ld_x, float p, int rounding, uint64_t seed,
-                    int scale_layout, void* stream) {
+                    int scale_layout, int elem, int stat, void* stream) {
   t_err.clear();
   int rc = check_common(x, T, D, ld_x);
   if (!rc) rc = check_out(q, "q");
@@ -438,9 +448,13 @@ static int fwd_like(int mode, const void* x, const void* gamma, void* q, void* s
     return fail(MXN_ERR_ARG, "rounding = %d", rounding);
   if (scale_layout != MXN_SCALES_ROWMAJOR && scale_layout != MXN_SCALES_MMA)
     return fail(MXN_ERR_ARG, "scale_layout = %d", scale_layout);
+  if (elem != MXN_ELEM_E4M3 && elem != MXN_ELEM_E2M1) return fail(MXN_ERR_ARG, "elem_format = %d", elem);
+  if (stat != MXN_STAT_ABSMAX && stat != MXN_STAT_SCALE_EXP) return fail(MXN_ERR_ARG, "statistic = %d", stat);
   if ((rc = injected())) return rc;
   if (T == 0) return MXN_OK;
   FwdArgs A{};
+  A.elem = elem == MXN_ELEM_E2M1 ? kElemE2M1 : kElemE4M3;
+  A.stat_exp = stat == MXN_STAT_SCALE_EXP;
   A.x = static_cast<const uint16_t*>(x);
   A.gamma = static_cast<const uint16_t*>(gamma);
   A.q = static_cast<uint8_t*>(q);
@@ -461,13 +475,42 @@ int mxnorm_fwd(const void* x, const void* gamma, void* q, void* scales, float* G
                int64_t D, int64_t ld_x, float p, int rounding, uint64_t seed, int scale_layout,
                void* stream) {
   return fwd_like(kModeMXNorm, x, gamma, q, scales, G_out, T, D, ld_x, p, rounding, seed,
-                  scale_layout, stream);
+                  scale_layout, MXN_ELEM_E4M3, MXN_STAT_ABSMAX, stream);
+}
+
+int mxnorm_fwd_ex(const void* x, const void* gamma, void* q, void* scales, float* G_out, int64_t T,
+                  int64_t D, int64_t ld_x, float p, int rounding, uint64_t seed, int scale_layout,
+                  int elem_format, int statistic, void* stream) {
+  return fwd_like(kModeMXNorm, x, gamma, q, scales, G_out, T, D, ld_x, p, rounding, seed,
+                  scale_layout, elem_format, statistic, stream);
 }
 
 int mxfp8_cast(const void* x, void* q, void* scales, int64_t T, int64_t D, int64_t ld_x,
                int rounding, uint64_t seed, int scale_layout, void* stream) {
   return fwd_like(kModeCast, x, nullptr, q, scales, nullptr, T, D, ld_x, 1.0f, rounding, seed,
-                  scale_layout, stream);
+                  scale_layout, MXN_ELEM_E4M3, MXN_STAT_ABSMAX, stream);
+}
+
+int mx_cast_ex(const void* x, const void* gain, void* q, void* scales, int64_t T, int64_t D,
+               int64_t ld_x, int rounding, uint64_t seed, int scale_layout, int elem_format,
+               void* stream) {
+  return fwd_like(kModeCast, x, gain, q, scales, nullptr, T, D, ld_x, 1.0f, rounding, seed,
+                  scale_layout, elem_format, MXN_STAT_ABSMAX, stream);
+}
+
+int mxnorm_fold_weight(const void* w, const void* gamma, void* q, void* scales, int64_t N,
+                       int64_t K, int64_t ld_w, int elem_format, int scale_layout, void* stream) {
+  t_err.clear();
+  if (!gamma && N != 0) return fail(MXN_ERR_ARG, "gamma is NULL (nothing to fold)");
+  return fwd_like(kModeCast, w, gamma, q, scales, nullptr, N, K, ld_w, 1.0f, MXN_ROUND_RNE, 0,
+                  scale_layout, elem_format, MXN_STAT_ABSMAX, stream);
+}
+
+size_t mxnorm_codes_bytes(int64_t T, int64_t D, int elem_format) {
+  if (T < 0 || D <= 0 || D % kBlock != 0) return 0;
+  if (elem_format == MXN_ELEM_E4M3) return (size_t)(T * D);
+  if (elem_format == MXN_ELEM_E2M1) return (size_t)(T * (D / 2));
+  return 0;
 }
 
 int rmsnorm_bf16(const void* x, const void* gamma, void* y, int64_t T, int64_t D, int64_t ld_x,

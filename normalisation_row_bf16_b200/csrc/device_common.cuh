@@ -245,6 +245,16 @@ __device__ __forceinline__ int e8m0_exponent_bits(uint32_t abits) {
   return max(e, -127);  // finite fp32 keeps e <= 120
 }
 
+// The same rule for E2M1 elements (largest magnitude 6 = 1.5 * 2^2): the
+// smallest e in [-127, 127] with a <= 6 * 2^e.
+__device__ __forceinline__ int e2m1_exponent_bits(uint32_t abits) {
+  if (abits >= 0x7F800000u) return 128;
+  const int ef = (int)(abits >> 23);
+  int e = ef - 127 - 2 + ((abits & 0x7FFFFFu) > 0x400000u ? 1 : 0);
+  if (ef == 0) e = -127;
+  return max(e, -127);
+}
+
 // ------------------------------------------------------------------ E4M3 cast
 
 // Two fp32 -> two E4M3 codes, round to nearest even, saturating finite; the
@@ -265,6 +275,24 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4_rn(float a, float b, float c, flo
       "mov.b32 %0, {l, h};\n\t}"
       : "=r"(r)
       : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
+
+// ------------------------------------------------------------------ E2M1 cast
+
+// Eight fp32 -> eight E2M1 codes (nearest even, saturating to +-6), packed
+// four bits each with the code of v[0] in bits 0..3 through v[7] in bits
+// 28..31 (cvt puts its first source in the high nibble of the byte).
+__device__ __forceinline__ uint32_t cvt_e2m1x8_rn(const float (&v)[8]) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
   return r;
 }
 
@@ -306,6 +334,28 @@ __device__ __forceinline__ float sr_e4m3_grid(float v, uint32_t r) {
     lo = truncf(a * 512.0f) * (1.0f / 512.0f);
     step = 1.0f / 512.0f;
     inv_step_2_32 = 2199023255552.0f;                 // 2^41
+  }
+  const float t = (a - lo) * inv_step_2_32;
+  const uint32_t thr = __float2uint_ru(t);
+  const float m = (r < thr) ? lo + step : lo;
+  return copysignf(m, v);
+}
+
+// The same on the E2M1 grid (|v| <= 6, which the rounded-up scale ensures):
+// one fraction bit from 1 up, step 1/2 below 1.
+__device__ __forceinline__ float sr_e2m1_grid(float v, uint32_t r) {
+  const float a = fabsf(v);
+  const uint32_t ab = __float_as_uint(a);
+  float lo, step, inv_step_2_32;
+  if (ab >= 0x3F800000u) {  // |v| >= 1: 1 fraction bit kept
+    lo = __uint_as_float(ab & 0xFFC00000u);
+    const uint32_t ebits = ab & 0x7F800000u;          // 2^E
+    step = __uint_as_float(ebits - (1u << 23));       // 2^(E-1)
+    inv_step_2_32 = __uint_as_float((uint32_t)(127 + 127 + 1 + 32) * (1u << 23) - ebits);  // 2^(33-E)
+  } else {                  // below 1: step 1/2
+    lo = truncf(a * 2.0f) * 0.5f;
+    step = 0.5f;
+    inv_step_2_32 = 8589934592.0f;                    // 2^33
   }
   const float t = (a - lo) * inv_step_2_32;
   const uint32_t thr = __float2uint_ru(t);

@@ -37,6 +37,9 @@
 namespace mxn {
 
 enum RowMode { kModeMXNorm = 0, kModeCast = 1, kModeRMSNorm = 2 };
+// Element formats of the MX codes: E4M3 (MXFP8, a byte per code) and E2M1
+// (MXFP4, two codes per byte, the even column in the low nibble).
+enum ElemFormat { kElemE4M3 = 0, kElemE2M1 = 1 };
 enum PMode { kP1 = 1, kP2 = 2, kP4 = 4, kPInf = 0, kPGeneral = 3 };
 
 // Threads per CTA the register budget is sized for: a thread holding 4 blocks
@@ -75,6 +78,8 @@ struct FwdArgs {
   uint32_t seed_lo, seed_hi;
   int scale_mma;          // scales in the tcgen05 128x4 layout
   int kp4;                // K rounded up to a multiple of 4 (MMA layout)
+  int elem;               // element format (kElemE4M3 / kElemE2M1; the kernel's template)
+  int stat_exp;           // MXNorm statistic from the blocks' power-of-two scales
 };
 
 // Byte offset of scale (row, k) in the tcgen05 block-scale layout.
@@ -224,16 +229,43 @@ __device__ __forceinline__ void issue_row_block(const uint16_t* x, const FwdCfg&
 // 8c + 4h .. 8c + 4h + 3 of the chunk c that slot j holds.  Returns the
 // scale byte.  y are the block's 32 fp32 values in slot order, a their
 // absmax (>= 0 or NaN).
-template <bool SR>
+template <bool SR, int ELEM>
 __device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a, int rot,
                                                   uint64_t idx0, uint32_t sk0, uint32_t sk1,
                                                   uint32_t (&qw)[8]) {
-  const int e_raw = e8m0_exponent_bits(__float_as_uint(a) & 0x7FFFFFFFu);
-  const bool nan_block = (e_raw == 128);     // NaN / inf in the block: codes 0x7F, scale 0xFF
+  const uint32_t abits = __float_as_uint(a) & 0x7FFFFFFFu;
+  const int e_raw = ELEM == kElemE2M1 ? e2m1_exponent_bits(abits) : e8m0_exponent_bits(abits);
+  const bool nan_block = (e_raw == 128);     // NaN / inf in the block: fixed codes, scale 0xFF
   const int e = nan_block ? 0 : e_raw;
   const float inv = exp2_int(-e);
   const float2 inv2 = make_float2(inv, inv);
-  if constexpr (!SR) {
+  if constexpr (ELEM == kElemE2M1) {
+    // qw[j] holds slot j's eight codes
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 t = mul2(make_float2(y[8 * sl + 2 * i], y[8 * sl + 2 * i + 1]), inv2);
+        v[2 * i] = t.x;
+        v[2 * i + 1] = t.y;
+      }
+      if constexpr (SR) {
+        const int c = (sl + rot) & 3;
+        const uint64_t ctr = (idx0 + (uint64_t)(c * 8)) >> 2;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint64_t cc = ctr + h;
+          const uint4 r = philox4x32_10(make_uint4((uint32_t)cc, (uint32_t)(cc >> 32), 0u, 0u), sk0, sk1);
+          v[4 * h] = sr_e2m1_grid(v[4 * h], r.x);
+          v[4 * h + 1] = sr_e2m1_grid(v[4 * h + 1], r.y);
+          v[4 * h + 2] = sr_e2m1_grid(v[4 * h + 2], r.z);
+          v[4 * h + 3] = sr_e2m1_grid(v[4 * h + 3], r.w);
+        }
+      }
+      qw[sl] = nan_block ? 0x77777777u : cvt_e2m1x8_rn(v);
+    }
+  } else if constexpr (!SR) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float2 v0 = mul2(make_float2(y[4 * i], y[4 * i + 1]), inv2);
@@ -257,8 +289,10 @@ __device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a,
       }
     }
   }
+  if constexpr (ELEM == kElemE4M3) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) qw[i] = nan_block ? 0x7F7F7F7Fu : qw[i];
+    for (int i = 0; i < 8; ++i) qw[i] = nan_block ? 0x7F7F7F7Fu : qw[i];
+  }
   return nan_block ? (uint8_t)0xFF : (uint8_t)(e + 127);
 }
 
@@ -271,6 +305,24 @@ __device__ __forceinline__ void store_codes(uint8_t* qp, const uint32_t (&qw)[8]
     asm volatile("st.global.cs.v2.b32 [%0], {%1, %2};" ::"l"(qp + ((j + rot) & 3) * 8),
                  "r"(qw[2 * j]), "r"(qw[2 * j + 1])
                  : "memory");
+}
+
+// E2M1 codes of a block (16 bytes): slot j's word goes to bytes
+// 4 * ((j + rot) & 3) .. + 3.
+__device__ __forceinline__ void store_codes_e2m1(uint8_t* qp, const uint32_t (&qw)[8], int rot) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    asm volatile("st.global.cs.b32 [%0], %1;" ::"l"(qp + ((j + rot) & 3) * 4), "r"(qw[j]) : "memory");
+}
+
+// The power-of-two scale 2^e of a block whose absmax has bf16 bits m, as bf16
+// bits (e by the rounded-up rule for the element format; 2^-127 is the bf16
+// subnormal 0x0040).  Infinity and NaN pass through.
+template <int ELEM>
+__device__ __forceinline__ uint32_t scale_pow2_bf16(uint32_t m) {
+  if (m >= 0x7F80u) return m;
+  const int e = ELEM == kElemE2M1 ? e2m1_exponent_bits(m << 16) : e8m0_exponent_bits(m << 16);
+  return e == -127 ? 0x0040u : (uint32_t)(e + 127) << 7;
 }
 
 // gamma for slot j of block k as 8 floats (in the order of the slot's words).
@@ -295,7 +347,7 @@ __host__ __device__ constexpr bool gamma_fp32(int tpr) { return tpr == 0 || tpr 
 // TPR: threads per row as a compile-time constant (32, 64, 128, 256), or 0
 // for rows of fewer than 32 blocks, where C.tpr (< 32) rows share a warp.
 // HG: gamma given (MXNorm, RMSNorm); its shared-memory format follows TPR.
-template <int MODE, int BPT, int TPR, bool SR, bool HG>
+template <int MODE, int BPT, int TPR, bool SR, bool HG, int ELEM>
 __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const FwdArgs A, const FwdCfg C) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tpr = TPR ? TPR : C.tpr;
@@ -314,7 +366,7 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C.bar_off) + (size_t)g * 2 * C.stages;
   uint64_t* empty = full + C.stages;
   float2* red = reinterpret_cast<float2*>(smem + C.red_off) + (size_t)g * 2 * kRedSlots;
-  constexpr bool has_gamma = (MODE != kModeCast) && HG;
+  constexpr bool has_gamma = HG;   // MXNorm's gain, RMSNorm's, or a cast's (folded weight)
   constexpr bool kGF32 = gamma_fp32(TPR);
 
   // Global row group, numbered group-major so that the groups of one row
@@ -470,7 +522,10 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
       // ------------------------------------------------- MXNorm / MXCast
       float sc = 1.0f;
       if constexpr (MODE == kModeMXNorm) {
-        const float G = row_pmean<BPT, TPR>(mb, A, C, redp, bar_id, wig, lane);
+        uint32_t mst[BPT];
+#pragma unroll
+        for (int b = 0; b < BPT; ++b) mst[b] = A.stat_exp ? scale_pow2_bf16<ELEM>(mb[b]) : mb[b];
+        const float G = row_pmean<BPT, TPR>(mst, A, C, redp, bar_id, wig, lane);
         sc = (G == 0.0f) ? 0.0f : __frcp_rn(G);
         if (valid && tg == 0 && A.G_out) A.G_out[row] = G;
       }
@@ -482,7 +537,7 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
         const int kk = k < C.K ? k : C.K - 1;          // in-range gamma reads
         float y[32];
         float a;
-        if constexpr (MODE == kModeMXNorm && has_gamma) {
+        if constexpr (has_gamma) {
           float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -511,9 +566,12 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
         }
         uint32_t qw[8];
         const uint64_t idx0 = (uint64_t)(row * (int64_t)C.D + (int64_t)k * kBlock);
-        const uint8_t code = quantise_block<SR>(y, a, rot, idx0, A.seed_lo, A.seed_hi, qw);
+        const uint8_t code = quantise_block<SR, ELEM>(y, a, rot, idx0, A.seed_lo, A.seed_hi, qw);
         if (blk) {
-          store_codes(A.q + row * (int64_t)C.D + (int64_t)k * kBlock, qw, rot);
+          if constexpr (ELEM == kElemE2M1)
+            store_codes_e2m1(A.q + row * (int64_t)(C.D / 2) + (int64_t)k * (kBlock / 2), qw, rot);
+          else
+            store_codes(A.q + row * (int64_t)C.D + (int64_t)k * kBlock, qw, rot);
           const int64_t so = A.scale_mma ? mma_scale_offset(row, k, A.kp4) : row * (int64_t)C.K + k;
           A.scales[so] = code;
         }
@@ -535,22 +593,22 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
 // row for up to 4 blocks each (rows of up to 128 blocks), 64..256 threads with
 // 4 blocks each beyond, a runtime segment width for rows under 32 blocks.
 // Each translation unit that calls this instantiates its own mode's kernels.
-template <int MODE, bool SR, bool HG>
+template <int MODE, bool SR, bool HG, int ELEM = kElemE4M3>
 const void* pick_fwd_shape(int bpt, int tpr) {
-  if (tpr < 32) return bpt == 1 ? (const void*)row_fwd_kernel<MODE, 1, 0, SR, HG> : nullptr;
+  if (tpr < 32) return bpt == 1 ? (const void*)row_fwd_kernel<MODE, 1, 0, SR, HG, ELEM> : nullptr;
   if (tpr == 32) {
     switch (bpt) {
-      case 1: return (const void*)row_fwd_kernel<MODE, 1, 32, SR, HG>;
-      case 2: return (const void*)row_fwd_kernel<MODE, 2, 32, SR, HG>;
-      case 4: return (const void*)row_fwd_kernel<MODE, 4, 32, SR, HG>;
+      case 1: return (const void*)row_fwd_kernel<MODE, 1, 32, SR, HG, ELEM>;
+      case 2: return (const void*)row_fwd_kernel<MODE, 2, 32, SR, HG, ELEM>;
+      case 4: return (const void*)row_fwd_kernel<MODE, 4, 32, SR, HG, ELEM>;
       default: return nullptr;
     }
   }
   if (bpt != 4) return nullptr;
   switch (tpr) {
-    case 64: return (const void*)row_fwd_kernel<MODE, 4, 64, SR, HG>;
-    case 128: return (const void*)row_fwd_kernel<MODE, 4, 128, SR, HG>;
-    case 256: return (const void*)row_fwd_kernel<MODE, 4, 256, SR, HG>;
+    case 64: return (const void*)row_fwd_kernel<MODE, 4, 64, SR, HG, ELEM>;
+    case 128: return (const void*)row_fwd_kernel<MODE, 4, 128, SR, HG, ELEM>;
+    case 256: return (const void*)row_fwd_kernel<MODE, 4, 256, SR, HG, ELEM>;
     default: return nullptr;
   }
 }

@@ -17,6 +17,8 @@ from . import build as _build
 
 RNE, SR = 0, 1
 SCALES_ROWMAJOR, SCALES_MMA = 0, 1
+ELEM = {"e4m3": 0, "e2m1": 1}
+STAT = {"absmax": 0, "scale_exp": 1}
 MXN_OK, MXN_ERR_ARG, MXN_ERR_UNSUPPORTED, MXN_ERR_CUDA, MXN_ERR_TIMEOUT = 0, -1, -2, -3, -4
 
 # Every symbol include/mxnorm.h declares, with its ctypes signature.
@@ -24,8 +26,13 @@ _P, _I64, _U64, _F32, _I32, _SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_uin
                                    ctypes.c_int, ctypes.c_size_t)
 SIGNATURES = {
     "mxnorm_scales_bytes": (_SZ, [_I64, _I64, _I32]),
+    "mxnorm_codes_bytes": (_SZ, [_I64, _I64, _I32]),
     "mxnorm_fwd": (_I32, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F32, _I32, _U64, _I32, _P]),
+    "mxnorm_fwd_ex": (_I32, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _F32, _I32, _U64, _I32, _I32, _I32,
+                             _P]),
     "mxfp8_cast": (_I32, [_P, _P, _P, _I64, _I64, _I64, _I32, _U64, _I32, _P]),
+    "mx_cast_ex": (_I32, [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _U64, _I32, _I32, _P]),
+    "mxnorm_fold_weight": (_I32, [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _I32, _P]),
     "rmsnorm_bf16": (_I32, [_P, _P, _P, _I64, _I64, _I64, _F32, _P]),
     "rmsnorm_then_mxcast": (_I32, [_P, _P, _F32, _P, _P, _P, _I64, _I64, _I64, _I32, _P]),
     "mxnorm_bwd": (_I32, [_P, _P, _P, _P, _P, _P, _I64, _I64, _P, _SZ, _P]),
@@ -101,9 +108,9 @@ def scales_bytes(T: int, D: int, layout: int = SCALES_ROWMAJOR) -> int:
     return int(lib().mxnorm_scales_bytes(T, D, layout))
 
 
-def _alloc_outputs(x, T, D, layout, q, scales):
+def _alloc_outputs(x, T, D, layout, q, scales, elem: str = "e4m3"):
     if q is None:
-        q = torch.empty(T, D, dtype=torch.uint8, device=x.device)
+        q = torch.empty(T, D // 2 if elem == "e2m1" else D, dtype=torch.uint8, device=x.device)
     if scales is None:
         n = scales_bytes(T, D, layout)
         scales = (torch.empty(T, D // 32, dtype=torch.uint8, device=x.device) if layout == SCALES_ROWMAJOR
@@ -132,6 +139,46 @@ def mxfp8_cast(x, rounding: int = RNE, seed: int = 0, scale_layout: int = SCALES
     q, scales = _alloc_outputs(x, T, D, scale_layout, q, scales)
     _check(lib().mxfp8_cast(_ptr(x), _ptr(q), _ptr(scales), T, D, ld, int(rounding),
                             ctypes.c_uint64(seed & (2**64 - 1)), int(scale_layout), _stream(stream)))
+    return q, scales
+
+
+def mxnorm_fwd_ex(x, gamma=None, p: float = 2.0, rounding: int = RNE, seed: int = 0,
+                  scale_layout: int = SCALES_ROWMAJOR, elem: str = "e4m3", stat: str = "absmax",
+                  q=None, scales=None, G=None, stream=None):
+    """MXNorm forward with an element format ("e4m3", or "e2m1": q uint8 [T, D/2],
+    two codes per byte) and a block statistic ("absmax", or "scale_exp")."""
+    T, D, ld = _rows_ld(x)
+    gamma = _bf16_vec(gamma, D)
+    q, scales = _alloc_outputs(x, T, D, scale_layout, q, scales, elem)
+    if G is None:
+        G = torch.empty(T, dtype=torch.float32, device=x.device)
+    _check(lib().mxnorm_fwd_ex(_ptr(x), _ptr(gamma), _ptr(q), _ptr(scales), _ptr(G), T, D, ld,
+                               float(p), int(rounding), ctypes.c_uint64(seed & (2**64 - 1)),
+                               int(scale_layout), ELEM[elem], STAT[stat], _stream(stream)))
+    return q, scales, G
+
+
+def mx_cast(x, gain=None, rounding: int = RNE, seed: int = 0, scale_layout: int = SCALES_ROWMAJOR,
+            elem: str = "e4m3", q=None, scales=None, stream=None):
+    """MX quantisation of x, or of x * gain along each row: (q, scales)."""
+    T, D, ld = _rows_ld(x)
+    gain = _bf16_vec(gain, D)
+    q, scales = _alloc_outputs(x, T, D, scale_layout, q, scales, elem)
+    _check(lib().mx_cast_ex(_ptr(x), _ptr(gain), _ptr(q), _ptr(scales), T, D, ld, int(rounding),
+                            ctypes.c_uint64(seed & (2**64 - 1)), int(scale_layout), ELEM[elem],
+                            _stream(stream)))
+    return q, scales
+
+
+def fold_weight(w, gamma, elem: str = "e4m3", scale_layout: int = SCALES_MMA, q=None, scales=None,
+                stream=None):
+    """MXNormLinear folding: MX codes and scales of w[n, k] * gamma[k], w [N, K]
+    one output feature per row (the GEMM's B operand)."""
+    N, K, ld = _rows_ld(w)
+    gamma = _bf16_vec(gamma, K)
+    q, scales = _alloc_outputs(w, N, K, scale_layout, q, scales, elem)
+    _check(lib().mxnorm_fold_weight(_ptr(w), _ptr(gamma), _ptr(q), _ptr(scales), N, K, ld,
+                                    ELEM[elem], int(scale_layout), _stream(stream)))
     return q, scales
 
 

@@ -3,7 +3,7 @@
 Tolerances (the numeric contract):
 * G: within 1e-6 relative of the oracle's long-double p-mean (exact for
   p = inf, where G is a maximum).
-* E8M0 scales and E4M3 codes (nearest-even and stochastic): bit-exact against
+* E8M0 scales and E4M3 / E2M1 codes (nearest-even and stochastic): bit-exact against
   the oracle re-run with the kernel's own G bits (two-stage parity: the kernel
   and the oracle add the p-mean terms in different orders, so the fp32 G may
   differ in its last bits; given the same G every later step is a sequence of
@@ -30,8 +30,9 @@ def to_np_u8(t):
     return t.detach().cpu().contiguous().numpy().view(np.uint8)
 
 
-def check_mxnorm_fwd(x_dev, g_dev, p, rounding, seed, q, s, G, rows=None, strict=True):
-    """Two-stage parity of an mxnorm_fwd result; returns a small report dict."""
+def check_mxnorm_fwd(x_dev, g_dev, p, rounding, seed, q, s, G, rows=None, strict=True,
+                     stat="absmax", fmt="e4m3"):
+    """Two-stage parity of an mxnorm_fwd(_ex) result; returns a small report dict."""
     x_cpu = x_dev.cpu()
     g_cpu = None if g_dev is None else g_dev.cpu()
     T = x_cpu.shape[0]
@@ -39,7 +40,8 @@ def check_mxnorm_fwd(x_dev, g_dev, p, rounding, seed, q, s, G, rows=None, strict
     qh = to_np_u8(q)[rows_np]
     sh = to_np_u8(s)[rows_np]
     Gh = G.detach().cpu().numpy()[rows_np]
-    q_own, s_own, G_ref = oracle.mxnorm_fwd(x_cpu, g_cpu, p, rows=rows_np, rounding=rounding, seed=seed)
+    q_own, s_own, G_ref = oracle.mxnorm_fwd_ex(x_cpu, g_cpu, p, rows=rows_np, rounding=rounding, seed=seed,
+                                               stat=stat, fmt=fmt)
     # stage (i): the statistic
     G_ref64 = G_ref.astype(np.float64)
     if np.isinf(p):
@@ -48,11 +50,12 @@ def check_mxnorm_fwd(x_dev, g_dev, p, rounding, seed, q, s, G, rows=None, strict
         rel = np.abs(Gh.astype(np.float64) - G_ref64) / np.where(G_ref64 > 0, G_ref64, 1.0)
         assert rel.max() <= G_RTOL, f"G relative error {rel.max():.3e} > {G_RTOL}"
     # stage (ii): codes and scales from the kernel's G
-    q_ref, s_ref, _ = oracle.mxnorm_fwd(x_cpu, g_cpu, p, rows=rows_np, G_in=Gh, rounding=rounding, seed=seed)
+    q_ref, s_ref, _ = oracle.mxnorm_fwd_ex(x_cpu, g_cpu, p, rows=rows_np, G_in=Gh, rounding=rounding,
+                                           seed=seed, stat=stat, fmt=fmt)
     bad_s = np.count_nonzero(s_ref != sh)
     bad_q = np.count_nonzero(q_ref != qh)
     assert bad_s == 0, f"{bad_s} E8M0 scales differ"
-    assert bad_q == 0, f"{bad_q} E4M3 codes differ"
+    assert bad_q == 0, f"{bad_q} {fmt} code bytes differ"
     report = {"rows": int(rows_np.size), "G_max_rel": 0.0 if np.isinf(p) else float(rel.max())}
     if strict:
         report["strict_scale_mismatch"] = int(np.count_nonzero(s_own != sh))
@@ -60,10 +63,11 @@ def check_mxnorm_fwd(x_dev, g_dev, p, rounding, seed, q, s, G, rows=None, strict
     return report
 
 
-def check_cast(x_dev, rounding, seed, q, s):
-    q_ref, s_ref = oracle.mxfp8_cast(x_dev.cpu(), rounding=rounding, seed=seed)
+def check_cast(x_dev, rounding, seed, q, s, gain_dev=None, fmt="e4m3"):
+    g = None if gain_dev is None else gain_dev.cpu()
+    q_ref, s_ref = oracle.mx_cast(x_dev.cpu(), g, rounding=rounding, seed=seed, fmt=fmt)
     assert np.array_equal(to_np_u8(s), s_ref), "E8M0 scales differ"
-    assert np.array_equal(to_np_u8(q), q_ref), "E4M3 codes differ"
+    assert np.array_equal(to_np_u8(q), q_ref), f"{fmt} codes differ"
 
 
 def bf16_ulp_distance(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
