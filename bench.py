@@ -377,10 +377,31 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
                                bwd_bytes(T, D, wsb.numel()), "row_bwd_kernel + dgamma_reduce_kernel")
     del dys, dxs, Gbs
 
+    # Variants on the same batch: MXFP4 codes, the scale-reuse statistic.
+    outs4 = [(torch.empty(T, D // 2, dtype=torch.uint8, device=dev),
+              torch.empty(T, D // 32, dtype=torch.uint8, device=dev),
+              torch.empty(T, dtype=torch.float32, device=dev)) for _ in range(n_sets)]
+    out["mxfp4_fwd"] = run_graph_leg(args, world, dev, barrier,
+                                     lambda i: ops.mxnorm_fwd_ex(xs[i % n_sets], g, p, elem="e2m1",
+                                                                 q=outs4[i % n_sets][0], scales=outs4[i % n_sets][1],
+                                                                 G=outs4[i % n_sets][2]),
+                                     fp4_bytes(T, D), "row_fwd_kernel<MXNorm, E2M1>")
+    del outs4
+    outs = [(torch.empty(T, D, dtype=torch.uint8, device=dev), torch.empty(T, D // 32, dtype=torch.uint8, device=dev),
+             torch.empty(T, dtype=torch.float32, device=dev)) for _ in range(n_sets)]
+    out["scale_reuse_fwd"] = run_graph_leg(args, world, dev, barrier,
+                                           lambda i: ops.mxnorm_fwd_ex(xs[i % n_sets], g, p, stat="scale_exp",
+                                                                       q=outs[i % n_sets][0], scales=outs[i % n_sets][1],
+                                                                       G=outs[i % n_sets][2]),
+                                           algorithmic_bytes(T, D), "row_fwd_kernel<MXNorm>, scale-exponent statistic")
+    del outs
+
     # Downstream block-scaled MXFP8 GEMM (MXNormLinear): the MXNorm output of
-    # an 8192 x 4096 N(0,1) batch times the fused QKV weight [4096 x 6144].
+    # an 8192 x 4096 N(0,1) batch times the fused QKV weight [4096 x 6144];
+    # the weight folding (gamma into W) and the norm -> GEMM pipeline.
     if D == 4096 and T % 128 == 0:
         out["gemm"] = run_gemm_leg(args, w, rank, world, dev, barrier)
+        out.update(run_linear_legs(args, w, rank, world, dev, barrier))
 
     if args.sweep:
         out["sweep"] = run_sweep(args, world, dev, barrier)
@@ -511,6 +532,63 @@ def run_gemm_leg(args, w, rank, world, dev, barrier):
                          "unit": "TFLOP/s", "frac": round(tflops / world / fp8_peak, 4),
                          "peak_source": f"{src} bf16 x 2 (nominal fp8/bf16 ratio)"},
             "kernel": "gemm_mxfp8_kernel (tcgen05 mxf8f6f4 block_scale, 128x256 tiles)"}
+
+
+def fp4_bytes(T, D):
+    # read x (2 B/elem), write E2M1 codes (1/2 B/elem) and scales (1/32); gamma, G
+    return int(T * D * 2 + T * D // 2 + T * (D // 32) + 2 * D + 4 * T)
+
+
+def run_linear_legs(args, w, rank, world, dev, barrier):
+    """MXNormLinear: folding gamma into the QKV weight, and one linear layer's
+    input path + GEMM as a pipeline (MXNorm -> GEMM vs RMSNorm -> MXCast -> GEMM)."""
+    import torch
+    import torch.distributed as dist
+    from normalisation_row_bf16_b200 import ops, synthetic
+
+    T, K, N, p = w["T"], w["D"], 6144, w["p"]
+    res = {}
+    wt = synthetic.gemm_weight(N, K, seed=rank, device=dev)
+    g = synthetic.gamma(K, seed=rank, device=dev)
+    n_w = max(2, math.ceil(3 * L2_BYTES / (N * K * 3)))
+    wts = [wt] + [wt.clone() for _ in range(n_w - 1)]
+    bqs = [torch.empty(N, K, dtype=torch.uint8, device=dev) for _ in range(n_w)]
+    bss = [torch.zeros(ops.scales_bytes(N, K, ops.SCALES_MMA), dtype=torch.uint8, device=dev) for _ in range(n_w)]
+    res["fold_weight"] = run_graph_leg(args, world, dev, barrier,
+                                       lambda i: ops.fold_weight(wts[i % n_w], g, q=bqs[i % n_w], scales=bss[i % n_w]),
+                                       N * K * 3 + N * (K // 32) + 2 * K, "row_fwd_kernel<Cast, gain>")
+    bq, bs = bqs[0], bss[0]
+    del wts, bqs[1:], bss[1:]
+
+    # pipeline: per step one batch x -> codes -> C, inputs and outputs rotating
+    n_s = 3
+    xs = [synthetic.activations(T, K, "normal", seed=rank + j, device=dev) for j in range(n_s)]
+    aqs = [torch.empty(T, K, dtype=torch.uint8, device=dev) for _ in range(n_s)]
+    ass = [torch.zeros(ops.scales_bytes(T, K, ops.SCALES_MMA), dtype=torch.uint8, device=dev) for _ in range(n_s)]
+    Gs = [torch.empty(T, dtype=torch.float32, device=dev) for _ in range(n_s)]
+    cs = [torch.empty(T, N, dtype=torch.bfloat16, device=dev) for _ in range(n_s)]
+    ytmp = torch.empty(T, K, dtype=torch.bfloat16, device=dev)
+    bq_u, bs_u = ops.mxfp8_cast(wt, scale_layout=ops.SCALES_MMA)
+
+    def mxnorm_step(i):
+        j = i % n_s
+        ops.mxnorm_fwd(xs[j], None, p, scale_layout=ops.SCALES_MMA, q=aqs[j], scales=ass[j], G=Gs[j])
+        ops.mxfp8_gemm(aqs[j], ass[j], bq, bs, T, N, K, c=cs[j])
+
+    def two_pass_step(i):
+        j = i % n_s
+        ops.rmsnorm_then_mxcast(xs[j], g, 1e-5, scale_layout=ops.SCALES_MMA, y_tmp=ytmp, q=aqs[j], scales=ass[j])
+        ops.mxfp8_gemm(aqs[j], ass[j], bq_u, bs_u, T, N, K, c=cs[j])
+
+    flops = 2.0 * T * N * K
+    for name, fn in (("pipeline_mxnorm_gemm", mxnorm_step), ("pipeline_rmsnorm_mxcast_gemm", two_pass_step)):
+        r = run_graph_leg(args, world, dev, barrier, fn, 0, name)
+        res[name] = {"ms": r["ms"], "steps": r["steps"],
+                     "TFLOPs_gemm_equiv": round(world * flops / (r["ms"] * 1e-3) / 1e12, 1),
+                     "kernels_per_step": 2 if name.startswith("pipeline_mxnorm") else 3}
+    res["pipeline_speedup"] = round(res["pipeline_rmsnorm_mxcast_gemm"]["ms"] /
+                                    res["pipeline_mxnorm_gemm"]["ms"], 4)
+    return res
 
 
 # ---------------------------------------------------------- reference arm

@@ -677,7 +677,7 @@ int mxfp8_gemm(const void* a_q, const void* a_s, const void* b_q, const void* b_
   DeviceInfo dev;
   if ((rc = device_info(&dev))) return rc;
   const char* why = "";
-  const int e = gemm_mxfp8_launch(a_q, a_s, b_q, b_s, c, (int)M, (int)N, (int)K, dev.status,
+  const int e = gemm_mxfp8_launch(a_q, a_s, b_q, b_s, c, (int)M, (int)N, (int)K, dev.sms, dev.status,
                                   static_cast<cudaStream_t>(stream), &why);
   if (e) return fail(MXN_ERR_CUDA, "mxfp8_gemm: %s", why);
   return MXN_OK;

@@ -6,20 +6,26 @@
 //   C[m, n] = sum_k A(m, k) * B(n, k),  A(m,k) = e4m3(a_q[m,k]) * 2^(a_s[m,k/32] - 127),
 //   B likewise, fp32 accumulation in tensor memory, bf16 output.
 //
-// One CTA computes a 128 x 256 tile of C:
-//  * a producer thread streams 128-element K stages of A (128 x 128 B) and B
-//    (256 x 128 B) into a 4-stage shared-memory ring with TMA tensor copies
-//    (128-byte swizzle, no multicast), and the stage's scale atoms (the
-//    128-row x 4-block, 512-byte tiles of the tcgen05 scale layout) with 1-D
-//    bulk copies;
-//  * an MMA thread copies each stage's scale atoms into tensor memory
-//    (tcgen05.cp 32x128b, replicated to the four lane quarters) and issues four
-//    tcgen05.mma.kind::mxf8f6f4.block_scale (M = 128, N = 256, K = 32 each),
-//    then tcgen05.commit frees the stage when those MMAs retire;
-//  * after the last stage the four warps read the fp32 accumulator out of
-//    tensor memory (tcgen05.ld 32x32b) and write bf16.
+// Persistent CTAs, one per SM, walk the 128 x 256 output tiles (tile t, then
+// t + gridDim.x, ...; M-tiles fastest, so the CTAs in flight share B tiles):
+//  * warp 0, one thread: the producer streams 128-element K stages of A
+//    (128 x 128 B) and B (256 x 128 B) into a 4-stage shared-memory ring with
+//    TMA tensor copies (128-byte swizzle, no multicast), and the stage's scale
+//    atoms (the 128-row x 4-block, 512-byte tiles of the tcgen05 scale layout)
+//    with 1-D bulk copies -- straight on into the next tile's stages;
+//  * warp 1, one thread: copies each stage's scale atoms into tensor memory
+//    (tcgen05.cp 32x128b, replicated to the four lane quarters), issues four
+//    tcgen05.mma.kind::mxf8f6f4.block_scale (M = 128, N = 256, K = 32 each)
+//    and frees the stage with tcgen05.commit; after a tile's last stage it
+//    commits "accumulator full", and before a tile's first MMA it waits for
+//    "accumulator empty";
+//  * warps 2..9: each reads its lane quarter and column half of the fp32
+//    accumulator (tcgen05.ld 32x32b, 128 columns) into registers, hands the
+//    accumulator back, and only then converts to bf16 and stores -- so the
+//    next tile's MMAs start after the tensor-memory read, not after the stores.
 // Every mbarrier wait is bounded; a wait that gives up records itself in the
-// device status word, and the CTA still frees its tensor memory.
+// device status word, every role stops, and the CTA waits (bounded) for its
+// copies and MMAs in flight before it frees its tensor memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -34,7 +40,8 @@ namespace {
 
 constexpr int kTileM = 128, kTileN = 256, kTileK = 128;  // K elements (= bytes) per stage
 constexpr int kStages = 4;
-constexpr int kThreads = 128;
+constexpr int kEpiWarps = 8;                     // 4 lane quarters x 2 column halves
+constexpr int kThreads = 64 + 32 * kEpiWarps;    // producer warp, MMA warp, epilogue warps
 constexpr uint32_t kABytes = kTileM * kTileK;    // 16 KiB
 constexpr uint32_t kBBytes = kTileN * kTileK;    // 32 KiB
 constexpr uint32_t kSfaBytes = 512;              // one 128 x 4 scale atom
@@ -51,7 +58,9 @@ struct Smem {
   uint8_t sfb[kStages][kSfbBytes];
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t acc_full;
+  uint64_t acc_full;                             // MMA -> epilogue (tcgen05.commit)
+  uint64_t acc_empty;                            // epilogue warps -> MMA
+  uint64_t mma_done;                             // every MMA of this CTA retired
   uint32_t tmem_base;
   uint32_t failed;
 };
@@ -108,7 +117,7 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 consecutive fp32 accumulator columns of this warp's 32 lanes.
+// 32 consecutive fp32 accumulator columns of this warp's 32 lanes (no wait).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -118,7 +127,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Orders every later use of r after the tensor-memory loads have landed: the
+// first call carries the wait, and each call rewrites its registers, so the
+// compiler cannot move a read of them above it.
+__device__ __forceinline__ void tmem_ld_fence(uint32_t (&r)[32], bool wait) {
+#define MXN_R32 "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), \
+                "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),      \
+                "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),     \
+                "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),     \
+                "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+  if (wait)
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : MXN_R32 :: "memory");
+  else
+    asm volatile("" : MXN_R32 :: "memory");
+#undef MXN_R32
+}
+
+__device__ __forceinline__ bool failed_flag(const Smem& S) {
+  return *reinterpret_cast<const volatile uint32_t*>(&S.failed) != 0;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -128,7 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x, nt = blockIdx.y;   // tile coordinates
+  const int m_tiles = M / kTileM;
+  const int n_tiles_all = m_tiles * (N / kTileN);
   const int n_k = K / kTileK;
   const int kp4 = K / 32;                       // scale columns (K % 128 == 0, so already a multiple of 4)
 
@@ -138,6 +167,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&S.empty[s], 1);
     }
     mbar_init(&S.acc_full, 1);
+    mbar_init(&S.acc_empty, kEpiWarps);
+    mbar_init(&S.mma_done, 1);
     S.failed = 0;
     fence_barrier_init();
   }
@@ -153,81 +184,129 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
 
-  int n_issued = 0;                             // producer: stages issued
-  if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------- producer
-    for (int kb = 0; kb < n_k; ++kb) {
-      const int s = kb % kStages;
-      const uint32_t ph = (uint32_t)((kb / kStages) & 1);
-      if (!mbar_wait_bounded(&S.empty[s], ph ^ 1u, status)) { atomicOr(&S.failed, 1u); break; }
-      mbar_arrive_expect_tx(&S.full[s], kStageTx);
-      tma_load_2d(S.a[s], &map_a, kb * kTileK, mt * kTileM, &S.full[s]);
-      tma_load_2d(S.b[s], &map_b, kb * kTileK, nt * kTileN, &S.full[s]);
-      // scale atoms: (row tile, 4-block group) -> 512 contiguous bytes
-      bulk_g2s_plain(S.sfa[s], a_s + ((size_t)mt * (kp4 / 4) + kb) * 512, kSfaBytes, &S.full[s]);
-      bulk_g2s_plain(S.sfb[s], b_s + ((size_t)(2 * nt) * (kp4 / 4) + kb) * 512, 512, &S.full[s]);
-      bulk_g2s_plain(S.sfb[s] + 512, b_s + ((size_t)(2 * nt + 1) * (kp4 / 4) + kb) * 512, 512, &S.full[s]);
-      n_issued = kb + 1;
-    }
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------------------- MMA
-    bool ok = true;
-    for (int kb = 0; kb < n_k && ok; ++kb) {
-      const int s = kb % kStages;
-      const uint32_t ph = (uint32_t)((kb / kStages) & 1);
-      if (!mbar_wait_bounded(&S.full[s], ph, status)) { atomicOr(&S.failed, 1u); ok = false; break; }
-      tc_fence_after();
-      const uint32_t sfa_col = kSfCol0 + (uint32_t)s * 12u, sfb_col = sfa_col + 4u;
-      // scale atoms -> tensor memory: 32 rows x 16 B each, 8-row core matrices 128 B apart
-      tmem_cp_sf(tmem + sfa_col, smem_desc(smem_u32(S.sfa[s]), 0, 128, 0));
-      tmem_cp_sf(tmem + sfb_col, smem_desc(smem_u32(S.sfb[s]), 0, 128, 0));
-      tmem_cp_sf(tmem + sfb_col + 4u, smem_desc(smem_u32(S.sfb[s] + 512), 0, 128, 0));
-      const uint32_t a0 = smem_u32(S.a[s]), b0 = smem_u32(S.b[s]);
-#pragma unroll
-      for (int k = 0; k < kTileK / 32; ++k) {
-        // 32 bytes further along the 128-byte swizzled rows; 8-row atoms 1024 B apart
-        const uint64_t ad = smem_desc(a0 + 32u * k, 16, 1024, 2);
-        const uint64_t bd = smem_desc(b0 + 32u * k, 16, 1024, 2);
-        mma_mxf8(tmem + kAccCol, ad, bd, instr_desc((uint32_t)k),
-                 (tmem + sfa_col) | ((uint32_t)k << 30), (tmem + sfb_col) | ((uint32_t)k << 30),
-                 (kb > 0 || k > 0) ? 1u : 0u);
+  uint32_t n_issued = 0;                        // producer: stages issued
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- producer
+      uint32_t g = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles_all && ok; t += gridDim.x) {
+        const int mt = t % m_tiles, nt = t / m_tiles;
+        for (int kb = 0; kb < n_k; ++kb, ++g) {
+          const int s = (int)(g % kStages);
+          const uint32_t ph = (g / kStages) & 1u;
+          if (!mbar_wait_bounded(&S.empty[s], ph ^ 1u, status) || failed_flag(S)) {
+            atomicOr(&S.failed, 1u);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&S.full[s], kStageTx);
+          tma_load_2d(S.a[s], &map_a, kb * kTileK, mt * kTileM, &S.full[s]);
+          tma_load_2d(S.b[s], &map_b, kb * kTileK, nt * kTileN, &S.full[s]);
+          // scale atoms: (row tile, 4-block group) -> 512 contiguous bytes
+          bulk_g2s_plain(S.sfa[s], a_s + ((size_t)mt * (kp4 / 4) + kb) * 512, kSfaBytes, &S.full[s]);
+          bulk_g2s_plain(S.sfb[s], b_s + ((size_t)(2 * nt) * (kp4 / 4) + kb) * 512, 512, &S.full[s]);
+          bulk_g2s_plain(S.sfb[s] + 512, b_s + ((size_t)(2 * nt + 1) * (kp4 / 4) + kb) * 512, 512, &S.full[s]);
+          n_issued = g + 1;
+        }
       }
-      tc_commit(&S.empty[s]);                    // stage free once these MMAs retire
     }
-    tc_commit(&S.acc_full);                       // accumulator complete (or the loop gave up)
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------- MMA
+      uint32_t g = 0, it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles_all && ok; t += gridDim.x, ++it) {
+        if (!mbar_wait_bounded(&S.acc_empty, (it & 1u) ^ 1u, status) || failed_flag(S)) {
+          atomicOr(&S.failed, 1u);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < n_k; ++kb, ++g) {
+          const int s = (int)(g % kStages);
+          const uint32_t ph = (g / kStages) & 1u;
+          if (!mbar_wait_bounded(&S.full[s], ph, status) || failed_flag(S)) {
+            atomicOr(&S.failed, 1u);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa_col = kSfCol0 + (uint32_t)s * 12u, sfb_col = sfa_col + 4u;
+          // scale atoms -> tensor memory: 32 rows x 16 B each, 8-row core matrices 128 B apart
+          tmem_cp_sf(tmem + sfa_col, smem_desc(smem_u32(S.sfa[s]), 0, 128, 0));
+          tmem_cp_sf(tmem + sfb_col, smem_desc(smem_u32(S.sfb[s]), 0, 128, 0));
+          tmem_cp_sf(tmem + sfb_col + 4u, smem_desc(smem_u32(S.sfb[s] + 512), 0, 128, 0));
+          const uint32_t a0 = smem_u32(S.a[s]), b0 = smem_u32(S.b[s]);
+#pragma unroll
+          for (int k = 0; k < kTileK / 32; ++k) {
+            // 32 bytes further along the 128-byte swizzled rows; 8-row atoms 1024 B apart
+            const uint64_t ad = smem_desc(a0 + 32u * k, 16, 1024, 2);
+            const uint64_t bd = smem_desc(b0 + 32u * k, 16, 1024, 2);
+            mma_mxf8(tmem + kAccCol, ad, bd, instr_desc((uint32_t)k),
+                     (tmem + sfa_col) | ((uint32_t)k << 30), (tmem + sfb_col) | ((uint32_t)k << 30),
+                     (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(&S.empty[s]);                // stage free once these MMAs retire
+        }
+        if (ok) tc_commit(&S.acc_full);          // the tile's accumulator is complete
+      }
+      tc_commit(&S.mma_done);                    // arrives once every MMA above has retired
+      if (!ok) tc_commit(&S.acc_full);           // wake the epilogue; it sees the failure
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;
+    const int quarter = warp & 3;                // tcgen05.ld reaches lanes 32 * (warp % 4) ..
+    const int half = e >> 2;                     // columns 128 * half ..
+    uint32_t it = 0;
+    for (int t = blockIdx.x; t < n_tiles_all; t += gridDim.x, ++it) {
+      const int mt = t % m_tiles, nt = t / m_tiles;
+      const bool got = mbar_wait_bounded(&S.acc_full, it & 1u, status);
+      tc_fence_after();
+      if (!got || failed_flag(S)) {
+        if (lane == 0) atomicOr(&S.failed, 1u);
+        break;
+      }
+      uint32_t r[4][32];
+      const uint32_t ta = tmem + kAccCol + (uint32_t)(half * 128) + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tmem_ld32(ta + 32u * j, r[j]);
+      tmem_ld_fence(r[0], true);
+#pragma unroll
+      for (int j = 1; j < 4; ++j) tmem_ld_fence(r[j], false);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.acc_empty);  // the MMA thread may overwrite the accumulator
+      const int row = mt * kTileM + quarter * 32 + lane;
+      uint16_t* crow = c + (size_t)row * N + (size_t)nt * kTileN + half * 128;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t o[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[j][2 * i]), __uint_as_float(r[j][2 * i + 1]));
+          o[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<uint4*>(crow + 32 * j + 8 * v) = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+      }
+    }
   }
 
-  // ------------------------------------------------------------ epilogue
-  __syncwarp();
-  const bool got = mbar_wait_bounded(&S.acc_full, 0, status);
-  tc_fence_after();
-  __syncthreads();
-  if (got && S.failed == 0) {
-    const int row = mt * kTileM + warp * 32 + lane;          // this thread's accumulator lane
-    uint16_t* crow = c + (size_t)row * N + (size_t)nt * kTileN;
-#pragma unroll 1
-    for (int cc = 0; cc < kTileN; cc += 32) {
-      uint32_t r[32];
-      tmem_ld32(tmem + kAccCol + (uint32_t)cc + ((uint32_t)(warp * 32) << 16), r);
-      uint32_t o[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-        o[i] = *reinterpret_cast<const uint32_t*>(&h);
-      }
-#pragma unroll
-      for (int v = 0; v < 4; ++v)
-        *reinterpret_cast<uint4*>(crow + cc + 8 * v) = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-    }
-  }
+  // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
+  if (warp == 1 && lane == 0) mbar_wait_bounded(&S.mma_done, 0, status);
   // After a wait gave up, leave no copy in flight: the producer waits (bounded)
   // for the last issued phase of every stage.
-  if (warp == 0 && lane == 0 && S.failed != 0)
-    for (int j = (n_issued > kStages ? n_issued - kStages : 0); j < n_issued; ++j)
-      mbar_wait_bounded(&S.full[j % kStages], (uint32_t)((j / kStages) & 1), status);
-  __syncwarp();
+  if (warp == 0 && lane == 0 && failed_flag(S))
+    for (uint32_t j = (n_issued > (uint32_t)kStages ? n_issued - kStages : 0); j < n_issued; ++j)
+      mbar_wait_bounded(&S.full[j % kStages], (j / kStages) & 1u, status);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   if (warp == 0)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
@@ -263,7 +342,7 @@ size_t gemm_mxfp8_smem_bytes() { return sizeof(Smem) + 1024; }
 
 // Launch: returns 0, or -1 (tensor map could not be encoded) / cuda error code.
 int gemm_mxfp8_launch(const void* a_q, const void* a_s, const void* b_q, const void* b_s, void* c, int M,
-                      int N, int K, unsigned* status, cudaStream_t stream, const char** why) {
+                      int N, int K, int sms, unsigned* status, cudaStream_t stream, const char** why) {
   CUtensorMap ma, mb;
   if (!make_map(&ma, a_q, M, K, kTileM) || !make_map(&mb, b_q, N, K, kTileN)) {
     *why = "cuTensorMapEncodeTiled failed";
@@ -272,7 +351,8 @@ int gemm_mxfp8_launch(const void* a_q, const void* a_s, const void* b_q, const v
   const size_t smem = sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(gemm_mxfp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) { *why = cudaGetErrorString(e); return (int)e; }
-  dim3 grid(M / kTileM, N / kTileN);
+  const int tiles = (M / kTileM) * (N / kTileN);
+  dim3 grid(tiles < sms ? tiles : sms);
   gemm_mxfp8_kernel<<<grid, kThreads, smem, stream>>>(ma, mb, static_cast<const uint8_t*>(a_s),
                                                       static_cast<const uint8_t*>(b_s),
                                                       static_cast<uint16_t*>(c), M, N, K, status);

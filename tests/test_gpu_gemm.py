@@ -79,3 +79,20 @@ def test_gemm_llama8b_qkv_sampled():
     jj = np.concatenate([rng.integers(0, N, 400), [0, N - 1, 255, 256]])
     _check(aq, a_s, bq, b_s, c, ii, jj)
     assert torch.isfinite(c.float()).all()
+
+
+@pytest.mark.parametrize("M,N,K", [(4352, 2560, 512), (128 * 149, 256, 256), (256, 256 * 3, 2048)])
+def test_gemm_persistent_uneven_tiles_sampled(M, N, K):
+    """Tile counts that do not divide evenly over the persistent CTAs (340 and
+    149 tiles on 148 SMs, and fewer tiles than SMs); every tile sampled."""
+    aq, a_s_mma, a_s, bq, b_s_mma, b_s = _operands(M, N, K, seed=M + 7)
+    c = ops.mxfp8_gemm(aq, a_s_mma, bq, b_s_mma, M, N, K)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(M)
+    mt, nt = M // 128, N // 256
+    ti, tj = np.meshgrid(np.arange(mt), np.arange(nt), indexing="ij")
+    ii = (ti.ravel() * 128 + rng.integers(0, 128, ti.size))
+    jj = (tj.ravel() * 256 + rng.integers(0, 256, tj.size))
+    ii = np.concatenate([ii, [0, M - 1]])
+    jj = np.concatenate([jj, [N - 1, 0]])
+    _check(aq, a_s, bq, b_s, c, ii, jj)
