@@ -301,15 +301,30 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8_rn(const float (&v)[8]) {
 // Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, SC'11): each round
 // multiplies words 0 and 2 by fixed odd constants, swaps the halves and xors
 // in the round key; the key advances by the Weyl constants between rounds.
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
-  constexpr uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
-  constexpr uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+//
+// The round keys depend on the seed only, so a kernel builds them once
+// (PhiloxKeys) and every call xors them in.
+struct PhiloxKeys {
+  uint32_t k0[10], k1[10];
+};
+
+__device__ __forceinline__ PhiloxKeys philox_keys(uint32_t seed_lo, uint32_t seed_hi) {
+  PhiloxKeys K;
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    if (r > 0) { k0 += W0; k1 += W1; }
-    const uint32_t hi0 = __umulhi(M0, c.x), lo0 = M0 * c.x;
-    const uint32_t hi1 = __umulhi(M1, c.z), lo1 = M1 * c.z;
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    K.k0[r] = seed_lo + (uint32_t)r * 0x9E3779B9u;
+    K.k1[r] = seed_hi + (uint32_t)r * 0xBB67AE85u;
+  }
+  return K;
+}
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys& K) {
+  constexpr uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = (uint64_t)M0 * c.x, p1 = (uint64_t)M1 * c.z;
+    c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ K.k0[r], (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ K.k1[r],
+                   (uint32_t)p0);
   }
   return c;
 }
@@ -317,27 +332,25 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
 // Stochastic rounding of v (|v| <= 448, finite) onto the E4M3 grid, returned
 // as the fp32 grid value (exact) with v's sign.  lo = the grid value at or
 // below |v|, step = grid spacing there; up iff r < (|v| - lo) / step * 2^32.
-// Every intermediate is exact in fp32: lo is |v| with its low mantissa bits
-// cleared (or a multiple of 2^-9 below 2^-6), |v| - lo is exact, and the
-// scaling by 2^32 / step is a power of two; for an integer r, r < t holds iff
-// r < ceil(t), and ceil(t) < 2^32.
+// From 2^-6 up the grid keeps 3 fraction bits, so lo is |v| with its 20 low
+// mantissa bits cleared and (|v| - lo) / step * 2^32 is exactly those 20 bits
+// times 2^12: an integer comparison, and lo + step an integer add on the bits
+// (a carry steps into the next binade).  Below 2^-6 (E4M3 subnormals, step
+// 2^-9, rare after the block scale) the same quantities in fp32: lo a multiple
+// of 2^-9, |v| - lo exact, the scaling by 2^41 a power of two; for an integer
+// r, r < t holds iff r < ceil(t), and ceil(t) < 2^32.
 __device__ __forceinline__ float sr_e4m3_grid(float v, uint32_t r) {
-  const float a = fabsf(v);
-  const uint32_t ab = __float_as_uint(a);
-  float lo, step, inv_step_2_32;
-  if (ab >= 0x3C800000u) {  // |v| >= 2^-6: 3 fraction bits kept
-    lo = __uint_as_float(ab & 0xFFF00000u);
-    const uint32_t ebits = ab & 0x7F800000u;          // 2^E
-    step = __uint_as_float(ebits - (3u << 23));       // 2^(E-3)
-    inv_step_2_32 = __uint_as_float((uint32_t)(127 + 127 + 3 + 32) * (1u << 23) - ebits);  // 2^(35-E)
-  } else {                  // subnormal range of E4M3: step 2^-9
-    lo = truncf(a * 512.0f) * (1.0f / 512.0f);
-    step = 1.0f / 512.0f;
-    inv_step_2_32 = 2199023255552.0f;                 // 2^41
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t ab = b & 0x7FFFFFFFu;
+  if (ab >= 0x3C800000u) {
+    const uint32_t low = ab & 0xFFFFFu;
+    const uint32_t up = (r < (low << 12)) ? 0x100000u : 0u;
+    return __uint_as_float(((ab & 0xFFF00000u) + up) | (b & 0x80000000u));
   }
-  const float t = (a - lo) * inv_step_2_32;
-  const uint32_t thr = __float2uint_ru(t);
-  const float m = (r < thr) ? lo + step : lo;
+  const float a = __uint_as_float(ab);
+  const float lo = truncf(a * 512.0f) * (1.0f / 512.0f);
+  const uint32_t thr = __float2uint_ru((a - lo) * 2199023255552.0f);   // 2^41
+  const float m = (r < thr) ? lo + (1.0f / 512.0f) : lo;
   return copysignf(m, v);
 }
 

@@ -231,7 +231,7 @@ __device__ __forceinline__ void issue_row_block(const uint16_t* x, const FwdCfg&
 // absmax (>= 0 or NaN).
 template <bool SR, int ELEM>
 __device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a, int rot,
-                                                  uint64_t idx0, uint32_t sk0, uint32_t sk1,
+                                                  uint64_t idx0, const PhiloxKeys& pk,
                                                   uint32_t (&qw)[8]) {
   const uint32_t abits = __float_as_uint(a) & 0x7FFFFFFFu;
   const int e_raw = ELEM == kElemE2M1 ? e2m1_exponent_bits(abits) : e8m0_exponent_bits(abits);
@@ -256,7 +256,7 @@ __device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a,
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const uint64_t cc = ctr + h;
-          const uint4 r = philox4x32_10(make_uint4((uint32_t)cc, (uint32_t)(cc >> 32), 0u, 0u), sk0, sk1);
+          const uint4 r = philox4x32_10(make_uint4((uint32_t)cc, (uint32_t)(cc >> 32), 0u, 0u), pk);
           v[4 * h] = sr_e2m1_grid(v[4 * h], r.x);
           v[4 * h + 1] = sr_e2m1_grid(v[4 * h + 1], r.y);
           v[4 * h + 2] = sr_e2m1_grid(v[4 * h + 2], r.z);
@@ -280,7 +280,7 @@ __device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a,
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const uint64_t cc = ctr + h;
-        const uint4 r = philox4x32_10(make_uint4((uint32_t)cc, (uint32_t)(cc >> 32), 0u, 0u), sk0, sk1);
+        const uint4 r = philox4x32_10(make_uint4((uint32_t)cc, (uint32_t)(cc >> 32), 0u, 0u), pk);
         const int i0 = sl * 8 + h * 4;
         const float2 v0 = mul2(make_float2(y[i0], y[i0 + 1]), inv2);
         const float2 v1 = mul2(make_float2(y[i0 + 2], y[i0 + 3]), inv2);
@@ -411,6 +411,7 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
   // A wait that gives up marks the kernel failed; threads then keep going
   // without waiting so every named barrier still completes (outputs garbage,
   // accesses in bounds).
+  const PhiloxKeys pkeys = philox_keys(A.seed_lo, A.seed_hi);   // used by stochastic rounding only
   bool ok = true;
   int par = 0;
   const int bar_id = 1 + g;
@@ -566,7 +567,7 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
         }
         uint32_t qw[8];
         const uint64_t idx0 = (uint64_t)(row * (int64_t)C.D + (int64_t)k * kBlock);
-        const uint8_t code = quantise_block<SR, ELEM>(y, a, rot, idx0, A.seed_lo, A.seed_hi, qw);
+        const uint8_t code = quantise_block<SR, ELEM>(y, a, rot, idx0, pkeys, qw);
         if (blk) {
           if constexpr (ELEM == kElemE2M1)
             store_codes_e2m1(A.q + row * (int64_t)(C.D / 2) + (int64_t)k * (kBlock / 2), qw, rot);
@@ -603,6 +604,19 @@ const void* pick_fwd_shape(int bpt, int tpr) {
       case 4: return (const void*)row_fwd_kernel<MODE, 4, 32, SR, HG, ELEM>;
       default: return nullptr;
     }
+  }
+  if constexpr (SR) {
+    // stochastic rounding: one block per thread up to 256 blocks per row
+    // (the Philox arithmetic wants warps, not long unrolled bodies)
+    if (bpt == 1) {
+      switch (tpr) {
+        case 64: return (const void*)row_fwd_kernel<MODE, 1, 64, SR, HG, ELEM>;
+        case 128: return (const void*)row_fwd_kernel<MODE, 1, 128, SR, HG, ELEM>;
+        case 256: return (const void*)row_fwd_kernel<MODE, 1, 256, SR, HG, ELEM>;
+        default: return nullptr;
+      }
+    }
+    if (bpt == 2) return tpr == 256 ? (const void*)row_fwd_kernel<MODE, 2, 256, SR, HG, ELEM> : nullptr;
   }
   if (bpt != 4) return nullptr;
   switch (tpr) {
