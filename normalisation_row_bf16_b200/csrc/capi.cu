@@ -367,7 +367,20 @@ int launch_fwd(int mode, bool sr, const FwdArgs& A, int64_t T, int D, int64_t ld
   a.status = dev.status;
   a.inv_K = 1.0f / (float)(D / kBlock);
   void* argv[] = {&a, &P.C};
-  cudaError_t e = cudaLaunchKernel(P.kernel, dim3(P.grid), dim3(P.threads), argv, P.smem, stream);
+  // Programmatic dependent launch: the kernel may start while the previous
+  // kernel in the stream drains; it waits (griddepcontrol.wait) before it
+  // reads or writes any tensor.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P.grid);
+  cfg.blockDim = dim3(P.threads);
+  cfg.dynamicSmemBytes = P.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelExC(&cfg, P.kernel, argv);
   if (e != cudaSuccess) return cuda_fail(e, "row_fwd_kernel launch");
   return MXN_OK;
 }

@@ -126,6 +126,15 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return p;
 }
 
+// Programmatic dependent launch: wait until the grids this one depends on in
+// stream order have completed and their writes are visible (a no-op when the
+// launch did not opt in), and let the next grid in the stream launch early
+// (its CTAs run once SMs free up, and wait in their own griddep_wait).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -98,7 +98,7 @@ __device__ __forceinline__ float2 row_sum2(float2 v, const RowCfg& C, float2* re
 }
 
 template <int NCT>
-__global__ void __launch_bounds__(CtaShape<NCT>::threads, NCT <= 128 ? 3 : 1)
+__global__ void __launch_bounds__(CtaShape<NCT>::threads, NCT <= 128 ? 2 : 1)
     row_bwd_kernel(const BwdArgs A, const RowCfg C) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* stage0 = smem;
@@ -139,72 +139,70 @@ __global__ void __launch_bounds__(CtaShape<NCT>::threads, NCT <= 128 ? 3 : 1)
 #pragma unroll
   for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
 
-  // x and dy stay in the stage: pass 1 reads them for the two row sums, pass 2
-  // reads them again for dx and the dgamma partials, and only then is the
-  // stage released.  That keeps the registers for the 32 dgamma accumulators.
+  // Each thread copies its x and dy blocks from the stage into registers and
+  // hands the stage back before any arithmetic, so the producer refills it
+  // while the row is reduced; G is fetched before the row's wait.  Products
+  // run as packed fp32 pairs.
   bool ok = true;
   int par = 0;
   int64_t it = 0;
   for (int64_t rb = blockIdx.x; rb < C.n_row_blocks; rb += gridDim.x, ++it, par ^= 1) {
     const int s = (int)(it % C.stages);
     const uint32_t ph = (uint32_t)((it / C.stages) & 1);
-    if (ok) ok = mbar_wait_bounded(&full[s], ph, A.status);
     const int64_t row = rb * C.rps + grp;
     const bool valid = row < C.T;
     const bool have = valid && mine;
+    const float G = have ? __ldg(A.G + row) : 0.0f;
+    if (ok) ok = mbar_wait_bounded(&full[s], ph, A.status);
     const uint8_t* sbase = stage0 + (size_t)s * C.stage_bytes;
     const uint32_t sx = smem_u32(sbase + (size_t)grp * C.row_bytes) + (uint32_t)k * 64u;
     const uint32_t sd = smem_u32(sbase + (size_t)(C.rps + grp) * C.row_bytes) + (uint32_t)k * 64u;
-
-    float2 part = make_float2(0.0f, 0.0f);  // (x . x, x . g)
-    if (have) {
+    uint32_t xa[16], da[16];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t off = (uint32_t)(((j + rot) & 3) * 16);
-        const uint4 a = lds128(sx + off), d = lds128(sd + off);
-        const uint32_t xa[4] = {a.x, a.y, a.z, a.w}, da[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t g2 = gw[4 * j + i];
-          const float x0 = bf16lo(xa[i]), x1 = bf16hi(xa[i]);
-          part.x = fmaf(x0, x0, part.x);
-          part.x = fmaf(x1, x1, part.x);
-          part.y = fmaf(x0, __fmul_rn(bf16lo(g2), bf16lo(da[i])), part.y);
-          part.y = fmaf(x1, __fmul_rn(bf16hi(g2), bf16hi(da[i])), part.y);
-        }
-      }
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t off = (uint32_t)(((j + rot) & 3) * 16);
+      uint4 a = make_uint4(0u, 0u, 0u, 0u), d = make_uint4(0u, 0u, 0u, 0u);
+      if (have) { a = lds128(sx + off); d = lds128(sd + off); }
+      xa[4 * j] = a.x; xa[4 * j + 1] = a.y; xa[4 * j + 2] = a.z; xa[4 * j + 3] = a.w;
+      da[4 * j] = d.x; da[4 * j + 1] = d.y; da[4 * j + 2] = d.z; da[4 * j + 3] = d.w;
     }
-    const float2 tot = row_sum2(part, C, red, grp, tg, lane, par);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+
+    float2 xx = make_float2(0.0f, 0.0f), xg = make_float2(0.0f, 0.0f);  // (x . x, x . g) halves
+#pragma unroll
+    for (int w = 0; w < 16; ++w) {
+      const float2 x2 = bf16x2_to_f2(xa[w]);
+      const float2 g2 = mul2(bf16x2_to_f2(gw[w]), bf16x2_to_f2(da[w]));
+      xx = fma2(x2, x2, xx);
+      xg = fma2(x2, g2, xg);
+    }
+    const float2 tot = row_sum2(make_float2(xx.x + xx.y, xg.x + xg.y), C, red, grp, tg, lane, par);
     if (have) {
-      const float G = __ldg(A.G + row);
       const bool live = (G != 0.0f) && (tot.x != 0.0f);
       const float invG = live ? __frcp_rn(G) : 0.0f;
       const float coef = live ? tot.y / tot.x : 0.0f;
+      const float2 ncoef2 = make_float2(-coef, -coef), invG2 = make_float2(invG, invG);
       uint16_t* dxrow = A.dx + row * (int64_t)C.D + (int64_t)k * kBlock;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint32_t off = (uint32_t)(((j + rot) & 3) * 16);
-        const uint4 a = lds128(sx + off), d = lds128(sd + off);
-        const uint32_t xa[4] = {a.x, a.y, a.z, a.w}, da[4] = {d.x, d.y, d.z, d.w};
         uint32_t o[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int w = 4 * j + i;
-          const float x0 = bf16lo(xa[i]), x1 = bf16hi(xa[i]);
-          const float d0 = bf16lo(da[i]), d1 = bf16hi(da[i]);
-          const float g0 = __fmul_rn(bf16lo(gw[w]), d0), g1 = __fmul_rn(bf16hi(gw[w]), d1);
-          const float r0 = __fmul_rn(fmaf(-x0, coef, g0), invG);
-          const float r1 = __fmul_rn(fmaf(-x1, coef, g1), invG);
-          const __nv_bfloat162 h = __floats2bfloat162_rn(r0, r1);
+          const float2 x2 = bf16x2_to_f2(xa[w]);
+          const float2 d2 = bf16x2_to_f2(da[w]);
+          const float2 g2 = mul2(bf16x2_to_f2(gw[w]), d2);
+          const float2 r = mul2(fma2(x2, ncoef2, g2), invG2);
+          const __nv_bfloat162 h = __floats2bfloat162_rn(r.x, r.y);
           o[i] = *reinterpret_cast<const uint32_t*>(&h);
-          acc[2 * w] = fmaf(__fmul_rn(d0, x0), invG, acc[2 * w]);
-          acc[2 * w + 1] = fmaf(__fmul_rn(d1, x1), invG, acc[2 * w + 1]);
+          const float2 a2 = fma2(mul2(d2, x2), invG2, make_float2(acc[2 * w], acc[2 * w + 1]));
+          acc[2 * w] = a2.x;
+          acc[2 * w + 1] = a2.y;
         }
         stg128_stream(dxrow + ((j + rot) & 3) * 8, make_uint4(o[0], o[1], o[2], o[3]));
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
   }
 
   if (A.partial != nullptr && mine) {

@@ -376,13 +376,19 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
   const int64_t rb_end = gg < C.ngt ? C.n_row_blocks : 0;
   const uint64_t pol = policy_evict_first();
   // The first row copies go out before anything else, so their DRAM latency
-  // overlaps the gamma set-up below.
+  // overlaps the gamma set-up below.  Inputs are read only after the grids
+  // this launch depends on have finished (programmatic dependent launch: the
+  // barrier set-up above the wait overlaps the previous kernel's tail).
   if (issuer) {
     for (int s = 0; s < C.stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], n_gwarps);
     }
     fence_barrier_init();
+  }
+  griddep_wait();
+  griddep_launch_dependents();
+  if (issuer) {
     for (int s = 0; s < C.stages; ++s) {
       const int64_t rb = gg + (int64_t)s * C.ngt;
       if (rb < rb_end) issue_row_block(A.x, C, rb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
