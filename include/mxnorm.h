@@ -250,8 +250,9 @@ int mxfp8_gemm(const void* a_q, const void* a_s, const void* b_q, const void* b_
  * the dgamma partial sums live in one 8 MiB scratch array inside this library
  * (2^21 fp32, allocated when a device loads the library, held until exit).
  * The call allocates nothing.  To fit the scratch it may launch fewer CTAs
- * than mxnorm_bwd (at most 2^21 / (rows per stage * D) of them); it returns
- * MXN_ERR_UNSUPPORTED if even one CTA's partial rows would not fit.
+ * than mxnorm_bwd (every active row group writes its partial rows of D fp32,
+ * at most 2^21 / D rows in all); it returns MXN_ERR_UNSUPPORTED if even one
+ * CTA's partial rows would not fit.
  * The first call on a device looks up the scratch array's device address
  * (cudaGetSymbolAddress); make that first call outside any stream capture.
  * Every call on a device shares the one scratch array: calls that may overlap

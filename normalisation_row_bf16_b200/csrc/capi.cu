@@ -97,20 +97,6 @@ int ilog2(int v) {
   return l;
 }
 
-// Launch plan for a row kernel: rows split into row blocks of rps rows, one
-// consumer thread per 32-element block (bpt blocks when K > 512), a ring of
-// `stages` shared-memory stages, a persistent grid of SMs x resident CTAs.
-struct Plan {
-  RowCfg C;
-  const void* kernel = nullptr;
-  int bpt = 1;
-  int threads = 0;
-  size_t smem = 0;
-  int grid = 0;
-};
-
-using KernelPicker = const void* (*)(int bpt, int nct);
-
 // Resident CTAs per SM of (kernel, threads, dynamic shared memory) on the
 // current device.  The first use of a combination sets the kernel's dynamic
 // shared-memory limit and queries the occupancy; later launches reuse both,
@@ -148,50 +134,23 @@ int occupancy(const void* kernel, int threads, size_t smem, int* occ) {
   return MXN_OK;
 }
 
-int plan_rows(int64_t T, int D, int64_t ld_x, int n_inputs, KernelPicker pick, int sms, Plan* P) {
-  RowCfg& C = P->C;
-  C.T = T;
-  C.ld_x = ld_x;
-  C.D = D;
-  C.K = D / kBlock;
-  P->bpt = C.K > kMaxConsumerThreads ? 2 : 1;
-  C.tpr = next_pow2((C.K + P->bpt - 1) / P->bpt);
-  C.log2_tpr = ilog2(C.tpr);
-  int nct = g_tuning.consumer_threads ? g_tuning.consumer_threads : 128;
-  if (nct < C.tpr) nct = C.tpr;
-  if (P->bpt == 2) nct = kMaxConsumerThreads;
-  C.rps = nct / C.tpr;
-  C.n_cwarps = nct / 32;
-  C.row_bytes = 2u * (uint32_t)D;
-  C.stage_bytes = (uint32_t)C.rps * C.row_bytes * (uint32_t)n_inputs;
-  int stages = g_tuning.stages;
-  if (!stages) {
-    stages = (int)(49152u / C.stage_bytes);
-    stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
-  }
-  C.stages = stages;
-  C.n_row_blocks = (T + C.rps - 1) / C.rps;
-  const size_t red = (C.tpr > 32) ? (size_t)2 * C.rps * kRedSlots * sizeof(float2) : 0;
-  P->smem = (size_t)stages * C.stage_bytes + (size_t)2 * stages * sizeof(uint64_t) + red;
-  P->threads = nct + 32;
-  P->kernel = pick(P->bpt, nct);
-  if (!P->kernel) return fail(MXN_ERR_UNSUPPORTED, "no kernel for D = %d", D);
-  if (P->smem > 227u * 1024u)
-    return fail(MXN_ERR_UNSUPPORTED, "row of %d elements needs %zu bytes of shared memory", D, P->smem);
-  int occ = 0;
-  int rc = occupancy(P->kernel, P->threads, P->smem, &occ);
-  if (rc) return rc;
-  if (occ < 1) return fail(MXN_ERR_UNSUPPORTED, "row kernel does not fit on an SM (D = %d)", D);
-  if (g_tuning.ctas_per_sm && g_tuning.ctas_per_sm < occ) occ = g_tuning.ctas_per_sm;
-  const int64_t g = (int64_t)sms * occ;
-  P->grid = (int)(C.n_row_blocks < g ? C.n_row_blocks : g);
-  return MXN_OK;
-}
-
-int launch(const Plan& P, void* args, cudaStream_t stream) {
-  void* argv[] = {args, const_cast<RowCfg*>(&P.C)};
-  cudaError_t e = cudaLaunchKernel(P.kernel, dim3(P.grid), dim3(P.threads), argv, P.smem, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "row kernel launch");
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream drains; every row kernel waits
+// (griddepcontrol.wait) before it reads or writes a tensor.
+int launch_pdl(const void* kernel, int grid, int threads, size_t smem, void** argv, cudaStream_t stream,
+               const char* what) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelExC(&cfg, kernel, argv);
+  if (e != cudaSuccess) return cuda_fail(e, what);
   return MXN_OK;
 }
 
@@ -345,16 +304,6 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int
   return MXN_OK;
 }
 
-const void* bwd_kernel(int bpt, int nct) {
-  if (bpt != 1) return nullptr;
-  switch (nct) {
-    case 128: return (const void*)row_bwd_kernel<128>;
-    case 256: return (const void*)row_bwd_kernel<256>;
-    case 512: return (const void*)row_bwd_kernel<512>;
-    default: return nullptr;
-  }
-}
-
 int launch_fwd(int mode, bool sr, const FwdArgs& A, int64_t T, int D, int64_t ld_x,
                cudaStream_t stream) {
   DeviceInfo dev;
@@ -367,22 +316,7 @@ int launch_fwd(int mode, bool sr, const FwdArgs& A, int64_t T, int D, int64_t ld
   a.status = dev.status;
   a.inv_K = 1.0f / (float)(D / kBlock);
   void* argv[] = {&a, &P.C};
-  // Programmatic dependent launch: the kernel may start while the previous
-  // kernel in the stream drains; it waits (griddepcontrol.wait) before it
-  // reads or writes any tensor.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(P.grid);
-  cfg.blockDim = dim3(P.threads);
-  cfg.dynamicSmemBytes = P.smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelExC(&cfg, P.kernel, argv);
-  if (e != cudaSuccess) return cuda_fail(e, "row_fwd_kernel launch");
-  return MXN_OK;
+  return launch_pdl(P.kernel, P.grid, P.threads, P.smem, argv, stream, "row_fwd_kernel launch");
 }
 
 int pmode_of(float p) {
@@ -393,8 +327,96 @@ int pmode_of(float p) {
   return kPGeneral;
 }
 
-int plan_bwd(int64_t T, int D, int sms, Plan* P) {
-  return plan_rows(T, D, D, 2, bwd_kernel, sms, P);
+// Launch plan of the backward row kernel (row_bwd.cuh).
+struct BwdPlan {
+  BwdCfg C;
+  const void* kernel = nullptr;
+  int threads = 0;
+  size_t smem = 0;
+  int grid = 0;
+  size_t partial_rows() const { return (size_t)C.ngt * (size_t)C.rps; }
+};
+
+// Rows of up to 256 blocks: one block per thread (tpr = K, several rows per
+// warp below 32 blocks); 257..512 blocks: 256 threads with two blocks each.
+// Row groups per CTA fill the register budget (512 threads, or 256 with two
+// blocks), one stage each by default; one CTA per SM.
+// max_partial_rows > 0 caps the groups that get rows (the allocation-free
+// entry point's scratch).
+int plan_bwd(int64_t T, int D, int sms, BwdPlan* P, int64_t max_partial_rows = 0) {
+  BwdCfg& C = P->C;
+  C = BwdCfg{};
+  C.T = T;
+  C.D = D;
+  C.K = D / kBlock;
+  int bpt;
+  if (C.K <= 256) { bpt = 1; C.tpr = next_pow2(C.K); }
+  else if (C.K <= 512) { bpt = 2; C.tpr = 256; }
+  else return fail(MXN_ERR_UNSUPPORTED, "mxnorm_bwd: D = %d > %d", D, kMaxBwdD);
+  C.log2_tpr = ilog2(C.tpr);
+  C.gthreads = C.tpr < 32 ? 32 : C.tpr;
+  C.rps = C.gthreads / C.tpr;
+  C.row_bytes = 2u * (uint32_t)D;
+  C.stage_bytes = 2u * (uint32_t)C.rps * C.row_bytes;
+  const int max_threads = bwd_max_threads(bpt);
+  int threads = g_tuning.consumer_threads ? g_tuning.consumer_threads : max_threads;
+  if (threads > max_threads) threads = max_threads;
+  int ng = threads / C.gthreads;
+  if (ng < 1) ng = 1;
+  if (C.tpr > 32 && ng > 15) ng = 15;  // named barriers 1..15
+  const size_t smem_cap = 227u * 1024u;
+  const size_t per_group_fixed = (size_t)2 * kRedSlots * sizeof(float2) + 16;
+  // One stage per group measured best on B200 (8192 x 4096: 47.4 us against
+  // 49.1 with two stages and 51.6 with three groups of two stages).
+  const int stages = g_tuning.stages ? g_tuning.stages : 1;
+  auto smem_of = [&](int n) {
+    return (size_t)n * stages * (C.stage_bytes + 2 * sizeof(uint64_t)) + (size_t)n * per_group_fixed + 16;
+  };
+  while (ng > 1 && smem_of(ng) > smem_cap) --ng;
+  if (smem_of(ng) > smem_cap)
+    return fail(MXN_ERR_UNSUPPORTED, "mxnorm_bwd: a row of %d elements does not fit in shared memory", D);
+  C.ng = ng;
+  C.stages = stages;
+  C.n_row_blocks = (T + C.rps - 1) / C.rps;
+  C.ring_off = 0;
+  C.bar_off = (uint32_t)align_up((size_t)ng * stages * C.stage_bytes, 16);
+  C.red_off = C.bar_off + (uint32_t)(ng * 2 * stages * sizeof(uint64_t));
+  P->smem = C.red_off + (size_t)ng * 2 * kRedSlots * sizeof(float2);
+  P->threads = ng * C.gthreads;
+  P->kernel = pick_bwd_shape(bpt, C.tpr);
+  if (!P->kernel) return fail(MXN_ERR_UNSUPPORTED, "mxnorm_bwd: no kernel for D = %d", D);
+  int occ = 0;
+  int rc = occupancy(P->kernel, P->threads, P->smem, &occ);
+  if (rc) return rc;
+  if (occ < 1) return fail(MXN_ERR_UNSUPPORTED, "mxnorm_bwd: row kernel does not fit on an SM (D = %d)", D);
+  if (g_tuning.ctas_per_sm && g_tuning.ctas_per_sm < occ) occ = g_tuning.ctas_per_sm;
+  int64_t ctas = (C.n_row_blocks + ng - 1) / ng;
+  if (ctas > (int64_t)sms * occ) ctas = (int64_t)sms * occ;
+  if (max_partial_rows > 0) {
+    const int64_t cap = max_partial_rows / ((int64_t)ng * C.rps);
+    if (cap < 1)
+      return fail(MXN_ERR_UNSUPPORTED, "%lld partial rows per CTA exceed the scratch",
+                  (long long)((int64_t)ng * C.rps));
+    if (ctas > cap) ctas = cap;
+  }
+  const int64_t R = (C.n_row_blocks + ctas * ng - 1) / (ctas * ng);
+  C.ngt = R > 0 ? (C.n_row_blocks + R - 1) / R : 0;
+  P->grid = (int)ctas;
+  return MXN_OK;
+}
+
+// Backward row kernel, then (when partial is set) the fixed-order dgamma sum.
+int launch_bwd(const BwdPlan& P, const BwdArgs& A, uint16_t* dgamma, cudaStream_t s) {
+  void* argv[] = {const_cast<BwdArgs*>(&A), const_cast<BwdCfg*>(&P.C)};
+  int rc = launch_pdl(P.kernel, P.grid, P.threads, P.smem, argv, s, "row_bwd_kernel launch");
+  if (rc) return rc;
+  if (A.partial) {
+    dgamma_reduce_kernel<<<(unsigned)((P.C.D + 31) / 32), dim3(32, 32), 0, s>>>(
+        A.partial, (int64_t)P.partial_rows(), P.C.D, dgamma);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "dgamma_reduce_kernel launch");
+  }
+  return MXN_OK;
 }
 
 // ----------------------------------------------- allocation-free backward
@@ -571,9 +593,9 @@ size_t mxnorm_bwd_workspace_size(int64_t T, int64_t D) {
   if (T <= 0 || D <= 0 || D % kBlock != 0 || D > kMaxBwdD) return 0;
   DeviceInfo dev;
   if (device_info(&dev)) return 0;
-  Plan P;
+  BwdPlan P;
   if (plan_bwd(T, (int)D, dev.sms, &P)) return 0;
-  return (size_t)P.grid * P.C.rps * (size_t)D * sizeof(float);
+  return P.partial_rows() * (size_t)D * sizeof(float);
 }
 
 int mxnorm_bwd(const void* x, const void* dy, const void* gamma, const float* G, void* dx,
@@ -593,9 +615,9 @@ int mxnorm_bwd(const void* x, const void* dy, const void* gamma, const float* G,
   if (T == 0) return MXN_OK;
   DeviceInfo dev;
   if ((rc = device_info(&dev))) return rc;
-  Plan P;
+  BwdPlan P;
   if ((rc = plan_bwd(T, (int)D, dev.sms, &P))) return rc;
-  const size_t need = (size_t)P.grid * P.C.rps * (size_t)D * sizeof(float);
+  const size_t need = P.partial_rows() * (size_t)D * sizeof(float);
   if (dgamma) {
     if (!workspace || !aligned16(workspace))
       return fail(MXN_ERR_ARG, "workspace is NULL or not 16-byte aligned");
@@ -610,15 +632,7 @@ int mxnorm_bwd(const void* x, const void* dy, const void* gamma, const float* G,
   A.dx = static_cast<uint16_t*>(dx);
   A.partial = dgamma ? static_cast<float*>(workspace) : nullptr;
   A.status = dev.status;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((rc = launch(P, &A, s))) return rc;
-  if (dgamma) {
-    dgamma_reduce_kernel<<<(unsigned)((D + 31) / 32), dim3(32, 32), 0, s>>>(
-        A.partial, (int64_t)P.grid * P.C.rps, (int)D, static_cast<uint16_t*>(dgamma));
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "dgamma_reduce_kernel launch");
-  }
-  return MXN_OK;
+  return launch_bwd(P, A, static_cast<uint16_t*>(dgamma), static_cast<cudaStream_t>(stream));
 }
 
 int mxnorm_bwd_noalloc(const void* x, const void* dy, const void* gamma, const float* G,
@@ -637,21 +651,14 @@ int mxnorm_bwd_noalloc(const void* x, const void* dy, const void* gamma, const f
   if (T == 0) return MXN_OK;
   DeviceInfo dev;
   if ((rc = device_info(&dev))) return rc;
-  Plan P;
-  if ((rc = plan_bwd(T, (int)D, dev.sms, &P))) return rc;
+  // Each active row group writes rps partial rows of D floats: plan no more
+  // of them than the scratch holds (the kernel is persistent, so fewer groups
+  // cover all rows).
+  BwdPlan P;
+  if ((rc = plan_bwd(T, (int)D, dev.sms, &P, dgamma ? (int64_t)(kNoAllocScratchFloats / (size_t)D) : 0)))
+    return rc;
   float* scratch = nullptr;
-  if (dgamma) {
-    if ((rc = noalloc_scratch(&scratch))) return rc;
-    // Each CTA writes rps partial rows of D floats: launch no more CTAs than
-    // the scratch holds (the kernel is persistent, so fewer CTAs cover all rows).
-    const int64_t per_cta = (int64_t)P.C.rps * D;
-    const int64_t max_ctas = (int64_t)kNoAllocScratchFloats / per_cta;
-    if (max_ctas < 1)
-      return fail(MXN_ERR_UNSUPPORTED,
-                  "mxnorm_bwd_noalloc: %lld partial floats per CTA exceed the %zu-float scratch",
-                  (long long)per_cta, kNoAllocScratchFloats);
-    if (P.grid > max_ctas) P.grid = (int)max_ctas;
-  }
+  if (dgamma && (rc = noalloc_scratch(&scratch))) return rc;
   BwdArgs A{};
   A.x = static_cast<const uint16_t*>(x);
   A.dy = static_cast<const uint16_t*>(dy);
@@ -660,15 +667,7 @@ int mxnorm_bwd_noalloc(const void* x, const void* dy, const void* gamma, const f
   A.dx = static_cast<uint16_t*>(dx);
   A.partial = scratch;
   A.status = dev.status;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((rc = launch(P, &A, s))) return rc;
-  if (dgamma) {
-    dgamma_reduce_kernel<<<(unsigned)((D + 31) / 32), dim3(32, 32), 0, s>>>(
-        scratch, (int64_t)P.grid * P.C.rps, (int)D, static_cast<uint16_t*>(dgamma));
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "dgamma_reduce_kernel launch");
-  }
-  return MXN_OK;
+  return launch_bwd(P, A, static_cast<uint16_t*>(dgamma), static_cast<cudaStream_t>(stream));
 }
 
 int mxfp8_gemm(const void* a_q, const void* a_s, const void* b_q, const void* b_s, void* c, int64_t M,

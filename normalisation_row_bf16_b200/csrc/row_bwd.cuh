@@ -8,40 +8,46 @@
 //     dgamma = sum over rows of dy * x / G
 // which is the exact gradient of x -> x * gamma / (c * rms(x)) at G = c * rms(x).
 //
-// Same pipeline as the forward (row_fwd.cuh): a producer thread streams the x
-// row and the dy row of each row block into a shared-memory stage with 1-D
-// bulk copies; a consumer thread owns one 32-column block of every row it
-// sees, so its dgamma partial sums stay in registers across rows.  At the end
-// every row group writes its partial row to the workspace; a second kernel adds
-// the partial rows in a fixed order (deterministic, no atomics).
+// Laid out like the forward (row_fwd.cuh):
+//  * a row group of tpr threads owns one row at a time (tpr = K up to 256
+//    blocks, one 32-column block per thread; rows of 257..512 blocks take 256
+//    threads with two blocks each; rows under 32 blocks share a warp), so a
+//    thread's dgamma partial sums for its columns stay in registers across
+//    every row the group sees;
+//  * each group has its own ring of stages (x rows, then dy rows) filled by
+//    1-D bulk copies that the group's first thread issues, completing on the
+//    group's own mbarriers;
+//  * a thread copies its x and dy blocks into registers and hands the stage
+//    back at once; G is fetched before the row's wait; products run as packed
+//    fp32 pairs; the two row sums (x . x, x . g) reduce with shuffles, plus
+//    shared memory and a named barrier when a row spans several warps.
+// At the end every active group writes its partial dgamma row(s) to the
+// workspace and dgamma_reduce_kernel adds them in a fixed order
+// (deterministic, no atomics).
 #pragma once
 
 #include "row_fwd.cuh"
 
 namespace mxn {
 
-constexpr int kMaxConsumerThreads = 512;
+// Threads per CTA the register budget is sized for: one block per thread
+// (x, dy, gamma and 32 accumulators in registers) fits 512 threads, two
+// blocks 256.
+__host__ __device__ constexpr int bwd_max_threads(int bpt) { return bpt == 1 ? 512 : 256; }
 
-// Launch shape of the backward: one consumer thread per 32-column block, rows
-// grouped rps per stage, one producer warp per CTA.
-struct RowCfg {
+struct BwdCfg {
   int64_t T;             // rows
-  int64_t ld_x;          // row stride of the input, elements
   int64_t n_row_blocks;  // ceil(T / rps)
-  int D, K;              // row length, blocks per row
-  int tpr, log2_tpr;     // consumer threads per row (power of two)
-  int rps;               // rows per stage
-  int stages;            // pipeline depth
-  int n_cwarps;          // consumer warps
+  int64_t ngt;           // row groups that get rows (<= groups in the grid)
+  int D, K;              // row length, MX blocks per row
+  int tpr, log2_tpr;     // threads per row (power of two)
+  int rps;               // rows per group and stage (> 1 only when tpr < 32)
+  int gthreads;          // threads per row group = max(tpr, 32)
+  int ng;                // row groups per CTA
+  int stages;            // ring depth per group
   uint32_t row_bytes;    // 2 * D
-  uint32_t stage_bytes;  // rps * row_bytes * 2 (x and dy)
-};
-
-// Resident CTAs per SM the register budget is sized for, by consumer threads
-// per CTA (each CTA adds one producer warp).
-template <int NCT>
-struct CtaShape {
-  static constexpr int threads = NCT + 32;
+  uint32_t stage_bytes;  // 2 * rps * row_bytes: rps x rows, then rps dy rows
+  uint32_t ring_off, bar_off, red_off;
 };
 
 struct BwdArgs {
@@ -50,139 +56,187 @@ struct BwdArgs {
   const uint16_t* gamma;  // bf16 [D] or null
   const float* G;         // fp32 [T]
   uint16_t* dx;           // bf16 [T, D]
-  float* partial;         // fp32 [gridDim.x * rps, D] or null (no dgamma)
+  float* partial;         // fp32 [ngt * rps, D] or null (no dgamma)
   unsigned* status;
 };
 
-__device__ __forceinline__ void produce_rows2(const uint16_t* x, const uint16_t* dy,
-                                              const RowCfg& C, uint8_t* stage0, uint64_t* full,
-                                              uint64_t* empty, unsigned* status) {
-  const uint64_t pol = policy_evict_first();
-  int64_t it = 0;
-  for (int64_t rb = blockIdx.x; rb < C.n_row_blocks; rb += gridDim.x, ++it) {
-    const int s = (int)(it % C.stages);
-    const uint32_t ph = (uint32_t)((it / C.stages) & 1);
-    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, status)) break;
-    const int64_t r0 = rb * C.rps;
-    const int nrows = (int)(C.T - r0 < (int64_t)C.rps ? C.T - r0 : (int64_t)C.rps);
-    mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)nrows * C.row_bytes);
-    uint8_t* dst = stage0 + (size_t)s * C.stage_bytes;
-    for (int r = 0; r < nrows; ++r) {
-      bulk_copy_g2s(dst + (size_t)r * C.row_bytes, x + (r0 + r) * C.ld_x, C.row_bytes, &full[s], pol);
-      bulk_copy_g2s(dst + (size_t)(C.rps + r) * C.row_bytes, dy + (r0 + r) * C.ld_x, C.row_bytes,
-                    &full[s], pol);
-    }
-  }
-  for (int64_t j = (it > C.stages ? it - C.stages : (int64_t)0); j < it; ++j)
-    mbar_wait_bounded(&full[j % C.stages], (uint32_t)((j / C.stages) & 1), status);
+// bf16 pair -> fp32 pair, as an opaque instruction pair: the second pass
+// converts its operands again instead of the compiler keeping the first
+// pass's 96 converted floats live (which would not fit the register budget).
+__device__ __forceinline__ float2 bf16x2_to_f2_again(uint32_t u) {
+  uint32_t lo, hi;
+  asm volatile("shl.b32 %0, %2, 16;\n\tand.b32 %1, %2, 0xFFFF0000;" : "=r"(lo), "=r"(hi) : "r"(u));
+  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
 }
 
-// Row sums of two quantities at once.
-__device__ __forceinline__ float2 row_sum2(float2 v, const RowCfg& C, float2* red, int grp, int tg,
-                                           int lane, int par) {
-  const int W = C.tpr < 32 ? C.tpr : 32;
+// Issue the bulk copies of row block rb (x rows, then dy rows) into `dst`.
+__device__ __forceinline__ void issue_bwd_block(const BwdArgs& A, const BwdCfg& C, int64_t rb,
+                                                uint8_t* dst, uint64_t* bar, uint64_t pol) {
+  const int64_t r0 = rb * C.rps;
+  const int nrows = (int)(C.T - r0 < (int64_t)C.rps ? C.T - r0 : (int64_t)C.rps);
+  mbar_arrive_expect_tx(bar, 2u * (uint32_t)nrows * C.row_bytes);
+  for (int r = 0; r < nrows; ++r) {
+    bulk_copy_g2s(dst + (size_t)r * C.row_bytes, A.x + (r0 + r) * (int64_t)C.D, C.row_bytes, bar, pol);
+    bulk_copy_g2s(dst + (size_t)(C.rps + r) * C.row_bytes, A.dy + (r0 + r) * (int64_t)C.D, C.row_bytes,
+                  bar, pol);
+  }
+}
+
+// The two row sums of a row group (segment of W lanes, then across warps).
+template <int TPR>
+__device__ __forceinline__ float2 row_sum2(float2 v, const BwdCfg& C, float2* red, int bar_id, int wig,
+                                           int lane) {
+  const int W = TPR ? (TPR < 32 ? TPR : 32) : C.tpr;
   v.x = seg_sum(v.x, W);
   v.y = seg_sum(v.y, W);
-  if (C.tpr > 32) {
-    const int nw = C.tpr >> 5;
-    float2* slot = red + (par * C.rps + grp) * kRedSlots;
-    if (lane == 0) slot[tg >> 5] = v;
-    named_barrier_sync(1 + grp, C.tpr);
+  if (TPR > 32) {
+    constexpr int nw = TPR > 32 ? TPR / 32 : 1;
+    if (lane == 0) red[wig] = v;
+    named_barrier_sync(bar_id, TPR);
     v = make_float2(0.0f, 0.0f);
+#pragma unroll
     for (int w = 0; w < nw; ++w) {
-      v.x += slot[w].x;
-      v.y += slot[w].y;
+      v.x += red[w].x;
+      v.y += red[w].y;
     }
   }
   return v;
 }
 
-template <int NCT>
-__global__ void __launch_bounds__(CtaShape<NCT>::threads, NCT <= 128 ? 2 : 1)
-    row_bwd_kernel(const BwdArgs A, const RowCfg C) {
+template <int BPT, int TPR>
+__global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const BwdArgs A, const BwdCfg C) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* stage0 = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)C.stages * C.stage_bytes);
-  uint64_t* empty = full + C.stages;
-  float2* red = reinterpret_cast<float2*>(empty + C.stages);
-
+  const int tpr = TPR ? TPR : C.tpr;
+  const int gthreads = TPR ? (TPR < 32 ? 32 : TPR) : 32;
   const int tid = threadIdx.x;
-  constexpr int ncons = NCT;
-  if (tid == 0) {
+  const int g = tid / gthreads;             // row group within the CTA
+  const int t = tid - g * gthreads;         // thread within the group
+  const int rs = TPR ? 0 : (t >> C.log2_tpr);  // row slot within the stage (rps > 1 only)
+  const int tg = t & (tpr - 1);             // thread within the row
+  const int lane = tid & 31;
+  const int wig = t >> 5;                   // warp within the group
+  const int n_gwarps = gthreads >> 5;
+  const bool issuer = (t == 0);
+
+  uint8_t* ring = smem + C.ring_off + (size_t)g * C.stages * C.stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C.bar_off) + (size_t)g * 2 * C.stages;
+  uint64_t* empty = full + C.stages;
+  float2* red = reinterpret_cast<float2*>(smem + C.red_off) + (size_t)g * 2 * kRedSlots;
+
+  const int64_t gg = (int64_t)g * gridDim.x + blockIdx.x;
+  const int64_t rb_end = gg < C.ngt ? C.n_row_blocks : 0;
+  const uint64_t pol = policy_evict_first();
+  if (issuer) {
     for (int s = 0; s < C.stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], C.n_cwarps);
+      mbar_init(&empty[s], n_gwarps);
     }
     fence_barrier_init();
   }
-  __syncthreads();
-  if (tid >= ncons) {
-    if (tid == ncons) produce_rows2(A.x, A.dy, C, stage0, full, empty, A.status);
-    return;
+  griddep_wait();
+  griddep_launch_dependents();
+  if (issuer) {
+    for (int s = 0; s < C.stages; ++s) {
+      const int64_t rb = gg + (int64_t)s * C.ngt;
+      if (rb < rb_end) issue_bwd_block(A, C, rb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
+    }
   }
 
-  const int lane = tid & 31;
-  const int grp = tid >> C.log2_tpr;
-  const int tg = tid & (C.tpr - 1);
-  const int k = tg;                       // one 32-column block per thread
-  const bool mine = k < C.K;
-  const int rot = (k >> 1) & 3;
-
-  uint32_t gw[16];
+  // gamma of this thread's blocks, in the thread's chunk order (ones when NULL)
+  const int rot = (tg >> 1) & 3;
+  uint32_t gw[BPT][16];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    uint4 v = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-    if (A.gamma != nullptr && mine) v = ldg128_nc(A.gamma + (size_t)k * kBlock + ((j + rot) & 3) * 8);
-    gw[4 * j] = v.x; gw[4 * j + 1] = v.y; gw[4 * j + 2] = v.z; gw[4 * j + 3] = v.w;
-  }
-  float acc[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-
-  // Each thread copies its x and dy blocks from the stage into registers and
-  // hands the stage back before any arithmetic, so the producer refills it
-  // while the row is reduced; G is fetched before the row's wait.  Products
-  // run as packed fp32 pairs.
-  bool ok = true;
-  int par = 0;
-  int64_t it = 0;
-  for (int64_t rb = blockIdx.x; rb < C.n_row_blocks; rb += gridDim.x, ++it, par ^= 1) {
-    const int s = (int)(it % C.stages);
-    const uint32_t ph = (uint32_t)((it / C.stages) & 1);
-    const int64_t row = rb * C.rps + grp;
-    const bool valid = row < C.T;
-    const bool have = valid && mine;
-    const float G = have ? __ldg(A.G + row) : 0.0f;
-    if (ok) ok = mbar_wait_bounded(&full[s], ph, A.status);
-    const uint8_t* sbase = stage0 + (size_t)s * C.stage_bytes;
-    const uint32_t sx = smem_u32(sbase + (size_t)grp * C.row_bytes) + (uint32_t)k * 64u;
-    const uint32_t sd = smem_u32(sbase + (size_t)(C.rps + grp) * C.row_bytes) + (uint32_t)k * 64u;
-    uint32_t xa[16], da[16];
+  for (int b = 0; b < BPT; ++b) {
+    const int k = tg + b * tpr;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t off = (uint32_t)(((j + rot) & 3) * 16);
-      uint4 a = make_uint4(0u, 0u, 0u, 0u), d = make_uint4(0u, 0u, 0u, 0u);
-      if (have) { a = lds128(sx + off); d = lds128(sd + off); }
-      xa[4 * j] = a.x; xa[4 * j + 1] = a.y; xa[4 * j + 2] = a.z; xa[4 * j + 3] = a.w;
-      da[4 * j] = d.x; da[4 * j + 1] = d.y; da[4 * j + 2] = d.z; da[4 * j + 3] = d.w;
+      uint4 v = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+      if (A.gamma != nullptr && k < C.K) v = ldg128_nc(A.gamma + (size_t)k * kBlock + ((j + rot) & 3) * 8);
+      gw[b][4 * j] = v.x; gw[b][4 * j + 1] = v.y; gw[b][4 * j + 2] = v.z; gw[b][4 * j + 3] = v.w;
+    }
+  }
+  float acc[BPT][32];
+#pragma unroll
+  for (int b = 0; b < BPT; ++b)
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[b][i] = 0.0f;
+  __syncthreads();                          // barrier set-up visible to every thread
+
+  bool ok = true;
+  int par = 0;
+  const int bar_id = 1 + g;
+  int64_t it = 0;
+  for (int64_t rb = gg; rb < rb_end; rb += C.ngt, ++it, par ^= 1) {
+    const int s = (int)(it % C.stages);
+    const uint32_t ph = (uint32_t)((it / C.stages) & 1);
+    const int64_t row = rb * C.rps + rs;
+    const bool valid = row < C.T;
+    const float G = valid ? __ldg(A.G + row) : 0.0f;
+    if (ok) ok = mbar_wait_bounded(&full[s], ph, A.status);
+    const uint8_t* st = ring + (size_t)s * C.stage_bytes;
+    const uint32_t sx = smem_u32(st + (size_t)rs * C.row_bytes);
+    const uint32_t sd = smem_u32(st + (size_t)(C.rps + rs) * C.row_bytes);
+
+    // ---- x and dy into registers, the stage straight back to the issuer
+    uint32_t xr[BPT][16], dr[BPT][16];
+#pragma unroll
+    for (int b = 0; b < BPT; ++b) {
+      const int k = tg + b * tpr;
+      const bool have = valid && k < C.K;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t off = (uint32_t)k * 64u + (uint32_t)(((j + rot) & 3) * 16);
+        uint4 a = make_uint4(0u, 0u, 0u, 0u), d = make_uint4(0u, 0u, 0u, 0u);
+        if (have) { a = lds128(sx + off); d = lds128(sd + off); }
+        xr[b][4 * j] = a.x; xr[b][4 * j + 1] = a.y; xr[b][4 * j + 2] = a.z; xr[b][4 * j + 3] = a.w;
+        dr[b][4 * j] = d.x; dr[b][4 * j + 1] = d.y; dr[b][4 * j + 2] = d.z; dr[b][4 * j + 3] = d.w;
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-
-    float2 xx = make_float2(0.0f, 0.0f), xg = make_float2(0.0f, 0.0f);  // (x . x, x . g) halves
-#pragma unroll
-    for (int w = 0; w < 16; ++w) {
-      const float2 x2 = bf16x2_to_f2(xa[w]);
-      const float2 g2 = mul2(bf16x2_to_f2(gw[w]), bf16x2_to_f2(da[w]));
-      xx = fma2(x2, x2, xx);
-      xg = fma2(x2, g2, xg);
+    // Refill: a one-warp row refills at once; a row of several warps after the
+    // row sum below, whose named barrier every warp reaches only after it has
+    // released the stage -- so the issuer's wait never holds up its warp.
+    const int64_t nrb = rb + (int64_t)C.stages * C.ngt;
+    if (TPR <= 32 && issuer && nrb < C.n_row_blocks) {
+      if (ok) ok = mbar_wait_bounded(&empty[s], ph, A.status);
+      if (ok) issue_bwd_block(A, C, nrb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
     }
-    const float2 tot = row_sum2(make_float2(xx.x + xx.y, xg.x + xg.y), C, red, grp, tg, lane, par);
-    if (have) {
-      const bool live = (G != 0.0f) && (tot.x != 0.0f);
-      const float invG = live ? __frcp_rn(G) : 0.0f;
-      const float coef = live ? tot.y / tot.x : 0.0f;
-      const float2 ncoef2 = make_float2(-coef, -coef), invG2 = make_float2(invG, invG);
+
+    // ---- pass 1: x . x and x . g (g = gamma * dy), and the dgamma partials
+    // dy * x / G (they need only G, which is known before the row arrives)
+    const float invG = (G != 0.0f) ? __frcp_rn(G) : 0.0f;
+    const float2 invG2 = make_float2(invG, invG);
+    float2 xx = make_float2(0.0f, 0.0f), xg = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int b = 0; b < BPT; ++b)
+#pragma unroll
+      for (int w = 0; w < 16; ++w) {
+        const float2 x2 = bf16x2_to_f2(xr[b][w]);
+        const float2 d2 = bf16x2_to_f2(dr[b][w]);
+        const float2 g2 = mul2(bf16x2_to_f2(gw[b][w]), d2);
+        xx = fma2(x2, x2, xx);
+        xg = fma2(x2, g2, xg);
+        const float2 a2 = fma2(mul2(d2, x2), invG2, make_float2(acc[b][2 * w], acc[b][2 * w + 1]));
+        acc[b][2 * w] = a2.x;
+        acc[b][2 * w + 1] = a2.y;
+      }
+    const float2 tot = row_sum2<TPR>(make_float2(xx.x + xx.y, xg.x + xg.y), C, red + par * kRedSlots,
+                                     bar_id, wig, lane);
+    if (TPR > 32 && issuer && nrb < C.n_row_blocks) {
+      if (ok) ok = mbar_wait_bounded(&empty[s], ph, A.status);
+      if (ok) issue_bwd_block(A, C, nrb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
+    }
+
+    // ---- pass 2: dx (zero for a row with G = 0 or x = 0)
+    const bool live = valid && (G != 0.0f) && (tot.x != 0.0f);
+    const float coef = live ? tot.y / tot.x : 0.0f;
+    const float sdx = live ? invG : 0.0f;
+    const float2 ncoef2 = make_float2(-coef, -coef), sdx2 = make_float2(sdx, sdx);
+#pragma unroll
+    for (int b = 0; b < BPT; ++b) {
+      const int k = tg + b * tpr;
+      const bool blk = valid && k < C.K;
       uint16_t* dxrow = A.dx + row * (int64_t)C.D + (int64_t)k * kBlock;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -190,28 +244,41 @@ __global__ void __launch_bounds__(CtaShape<NCT>::threads, NCT <= 128 ? 2 : 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int w = 4 * j + i;
-          const float2 x2 = bf16x2_to_f2(xa[w]);
-          const float2 d2 = bf16x2_to_f2(da[w]);
-          const float2 g2 = mul2(bf16x2_to_f2(gw[w]), d2);
-          const float2 r = mul2(fma2(x2, ncoef2, g2), invG2);
+          const float2 x2 = bf16x2_to_f2_again(xr[b][w]);
+          const float2 g2 = mul2(bf16x2_to_f2_again(gw[b][w]), bf16x2_to_f2_again(dr[b][w]));
+          const float2 r = mul2(fma2(x2, ncoef2, g2), sdx2);
           const __nv_bfloat162 h = __floats2bfloat162_rn(r.x, r.y);
           o[i] = *reinterpret_cast<const uint32_t*>(&h);
-          const float2 a2 = fma2(mul2(d2, x2), invG2, make_float2(acc[2 * w], acc[2 * w + 1]));
-          acc[2 * w] = a2.x;
-          acc[2 * w + 1] = a2.y;
         }
-        stg128_stream(dxrow + ((j + rot) & 3) * 8, make_uint4(o[0], o[1], o[2], o[3]));
+        if (blk) stg128_stream(dxrow + ((j + rot) & 3) * 8, make_uint4(o[0], o[1], o[2], o[3]));
       }
     }
   }
 
-  if (A.partial != nullptr && mine) {
-    float* prow = A.partial + ((int64_t)blockIdx.x * C.rps + grp) * C.D + (int64_t)k * kBlock;
+  // ---- this group's partial dgamma row (row slot rs)
+  if (A.partial != nullptr && gg < C.ngt) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float* p = prow + ((j + rot) & 3) * 8;
-      reinterpret_cast<float4*>(p)[0] = make_float4(acc[8 * j], acc[8 * j + 1], acc[8 * j + 2], acc[8 * j + 3]);
-      reinterpret_cast<float4*>(p)[1] = make_float4(acc[8 * j + 4], acc[8 * j + 5], acc[8 * j + 6], acc[8 * j + 7]);
+    for (int b = 0; b < BPT; ++b) {
+      const int k = tg + b * tpr;
+      if (k < C.K) {
+        float* prow = A.partial + ((int64_t)gg * C.rps + rs) * C.D + (int64_t)k * kBlock;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float* p = prow + ((j + rot) & 3) * 8;
+          reinterpret_cast<float4*>(p)[0] = make_float4(acc[b][8 * j], acc[b][8 * j + 1], acc[b][8 * j + 2],
+                                                        acc[b][8 * j + 3]);
+          reinterpret_cast<float4*>(p)[1] = make_float4(acc[b][8 * j + 4], acc[b][8 * j + 5],
+                                                        acc[b][8 * j + 6], acc[b][8 * j + 7]);
+        }
+      }
+    }
+  }
+  // Leave no copy in flight: the issuer waits for the last phase of every stage
+  // it filled (already complete unless a wait gave up above).
+  if (issuer && !ok) {
+    for (int s = 0; s < C.stages; ++s) {
+      const int64_t last_it = it - 1 - ((it - 1 - s) % C.stages + C.stages) % C.stages;
+      if (last_it >= 0) mbar_wait_bounded(&full[s], (uint32_t)((last_it / C.stages) & 1), A.status);
     }
   }
 }
@@ -234,6 +301,20 @@ __global__ void __launch_bounds__(1024) dgamma_reduce_kernel(const float* partia
     for (int i = 0; i < 32; ++i) t += sh[i][tx];
     const __nv_bfloat16 h = __float2bfloat16_rn(t);
     dgamma[j] = *reinterpret_cast<const uint16_t*>(&h);
+  }
+}
+
+// The instantiation for (blocks per thread, threads per row).
+inline const void* pick_bwd_shape(int bpt, int tpr) {
+  if (bpt == 2) return tpr == 256 ? (const void*)row_bwd_kernel<2, 256> : nullptr;
+  if (bpt != 1) return nullptr;
+  if (tpr < 32) return (const void*)row_bwd_kernel<1, 0>;
+  switch (tpr) {
+    case 32: return (const void*)row_bwd_kernel<1, 32>;
+    case 64: return (const void*)row_bwd_kernel<1, 64>;
+    case 128: return (const void*)row_bwd_kernel<1, 128>;
+    case 256: return (const void*)row_bwd_kernel<1, 256>;
+    default: return nullptr;
   }
 }
 
