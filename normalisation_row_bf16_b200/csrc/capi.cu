@@ -369,8 +369,10 @@ int plan_bwd(int64_t T, int D, int sms, BwdPlan* P, int64_t max_partial_rows = 0
   // One stage per group measured best on B200 (8192 x 4096: 47.4 us against
   // 49.1 with two stages and 51.6 with three groups of two stages).
   const int stages = g_tuning.stages ? g_tuning.stages : 1;
+  C.gamma_bytes = (uint32_t)align_up(2u * (uint32_t)D, 128);
   auto smem_of = [&](int n) {
-    return (size_t)n * stages * (C.stage_bytes + 2 * sizeof(uint64_t)) + (size_t)n * per_group_fixed + 16;
+    return (size_t)C.gamma_bytes + (size_t)n * stages * (C.stage_bytes + 2 * sizeof(uint64_t)) +
+           (size_t)n * per_group_fixed + 16;
   };
   while (ng > 1 && smem_of(ng) > smem_cap) --ng;
   if (smem_of(ng) > smem_cap)
@@ -378,8 +380,8 @@ int plan_bwd(int64_t T, int D, int sms, BwdPlan* P, int64_t max_partial_rows = 0
   C.ng = ng;
   C.stages = stages;
   C.n_row_blocks = (T + C.rps - 1) / C.rps;
-  C.ring_off = 0;
-  C.bar_off = (uint32_t)align_up((size_t)ng * stages * C.stage_bytes, 16);
+  C.ring_off = C.gamma_bytes;
+  C.bar_off = (uint32_t)align_up(C.ring_off + (size_t)ng * stages * C.stage_bytes, 16);
   C.red_off = C.bar_off + (uint32_t)(ng * 2 * stages * sizeof(uint64_t));
   P->smem = C.red_off + (size_t)ng * 2 * kRedSlots * sizeof(float2);
   P->threads = ng * C.gthreads;

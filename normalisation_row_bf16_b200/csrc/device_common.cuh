@@ -154,6 +154,14 @@ __device__ __forceinline__ void stg128_stream(void* p, uint4 v) {
                : "memory");
 }
 
+// A 4-byte read-only global load that stays where it is written (volatile), so
+// its latency overlaps what follows instead of being moved next to its use.
+__device__ __forceinline__ float ldg_f32_early(const float* p) {
+  float v;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ uint4 ldg128_nc(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];"

@@ -47,6 +47,7 @@ struct BwdCfg {
   int stages;            // ring depth per group
   uint32_t row_bytes;    // 2 * D
   uint32_t stage_bytes;  // 2 * rps * row_bytes: rps x rows, then rps dy rows
+  uint32_t gamma_bytes;  // gamma (or ones) in shared memory, slot order
   uint32_t ring_off, bar_off, red_off;
 };
 
@@ -142,18 +143,17 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
     }
   }
 
-  // gamma of this thread's blocks, in the thread's chunk order (ones when NULL)
+  // gamma (ones when NULL) into shared memory once per CTA in slot order: the
+  // 16 bytes that match x chunk slot j of block k at (j * K + k) * 16, so a
+  // warp's reads of one slot fall on consecutive words (registers stay free
+  // for x, dy and the dgamma sums).
   const int rot = (tg >> 1) & 3;
-  uint32_t gw[BPT][16];
-#pragma unroll
-  for (int b = 0; b < BPT; ++b) {
-    const int k = tg + b * tpr;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint4 v = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-      if (A.gamma != nullptr && k < C.K) v = ldg128_nc(A.gamma + (size_t)k * kBlock + ((j + rot) & 3) * 8);
-      gw[b][4 * j] = v.x; gw[b][4 * j + 1] = v.y; gw[b][4 * j + 2] = v.z; gw[b][4 * j + 3] = v.w;
-    }
+  for (int i = tid; i < C.K * 4; i += blockDim.x) {
+    const int k = i >> 2, j = i & 3;
+    const int c = (j + (k >> 1)) & 3;
+    uint4 v = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    if (A.gamma != nullptr) v = ldg128_nc(A.gamma + (size_t)k * kBlock + c * 8);
+    *reinterpret_cast<uint4*>(smem + ((size_t)j * C.K + k) * 16) = v;
   }
   float acc[BPT][32];
 #pragma unroll
@@ -166,12 +166,16 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
   int par = 0;
   const int bar_id = 1 + g;
   int64_t it = 0;
+  // G of the group's next row is loaded one row ahead.
+  float G_next = (gg < rb_end && gg * C.rps + rs < C.T) ? ldg_f32_early(A.G + gg * C.rps + rs) : 0.0f;
   for (int64_t rb = gg; rb < rb_end; rb += C.ngt, ++it, par ^= 1) {
     const int s = (int)(it % C.stages);
     const uint32_t ph = (uint32_t)((it / C.stages) & 1);
     const int64_t row = rb * C.rps + rs;
     const bool valid = row < C.T;
-    const float G = valid ? __ldg(A.G + row) : 0.0f;
+    const float G = G_next;
+    const int64_t row_n = (rb + C.ngt) * C.rps + rs;
+    G_next = (rb + C.ngt < rb_end && row_n < C.T) ? ldg_f32_early(A.G + row_n) : 0.0f;
     if (ok) ok = mbar_wait_bounded(&full[s], ph, A.status);
     const uint8_t* st = ring + (size_t)s * C.stage_bytes;
     const uint32_t sx = smem_u32(st + (size_t)rs * C.row_bytes);
@@ -209,18 +213,26 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
     const float2 invG2 = make_float2(invG, invG);
     float2 xx = make_float2(0.0f, 0.0f), xg = make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int b = 0; b < BPT; ++b)
+    for (int b = 0; b < BPT; ++b) {
+      const int kk = (tg + b * tpr) < C.K ? tg + b * tpr : C.K - 1;
 #pragma unroll
-      for (int w = 0; w < 16; ++w) {
-        const float2 x2 = bf16x2_to_f2(xr[b][w]);
-        const float2 d2 = bf16x2_to_f2(dr[b][w]);
-        const float2 g2 = mul2(bf16x2_to_f2(gw[b][w]), d2);
-        xx = fma2(x2, x2, xx);
-        xg = fma2(x2, g2, xg);
-        const float2 a2 = fma2(mul2(d2, x2), invG2, make_float2(acc[b][2 * w], acc[b][2 * w + 1]));
-        acc[b][2 * w] = a2.x;
-        acc[b][2 * w + 1] = a2.y;
+      for (int j = 0; j < 4; ++j) {
+        const uint4 gv4 = lds128(smem_u32(smem + ((size_t)j * C.K + kk) * 16));
+        const uint32_t gv[4] = {gv4.x, gv4.y, gv4.z, gv4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int w = 4 * j + i;
+          const float2 x2 = bf16x2_to_f2(xr[b][w]);
+          const float2 d2 = bf16x2_to_f2(dr[b][w]);
+          const float2 g2 = mul2(bf16x2_to_f2(gv[i]), d2);
+          xx = fma2(x2, x2, xx);
+          xg = fma2(x2, g2, xg);
+          const float2 a2 = fma2(mul2(d2, x2), invG2, make_float2(acc[b][2 * w], acc[b][2 * w + 1]));
+          acc[b][2 * w] = a2.x;
+          acc[b][2 * w + 1] = a2.y;
+        }
       }
+    }
     const float2 tot = row_sum2<TPR>(make_float2(xx.x + xx.y, xg.x + xg.y), C, red + par * kRedSlots,
                                      bar_id, wig, lane);
     if (TPR > 32 && issuer && nrb < C.n_row_blocks) {
@@ -240,12 +252,15 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
       uint16_t* dxrow = A.dx + row * (int64_t)C.D + (int64_t)k * kBlock;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
+        const int kk = k < C.K ? k : C.K - 1;
+        const uint4 gv4 = lds128(smem_u32(smem + ((size_t)j * C.K + kk) * 16));
+        const uint32_t gv[4] = {gv4.x, gv4.y, gv4.z, gv4.w};
         uint32_t o[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int w = 4 * j + i;
           const float2 x2 = bf16x2_to_f2_again(xr[b][w]);
-          const float2 g2 = mul2(bf16x2_to_f2_again(gw[b][w]), bf16x2_to_f2_again(dr[b][w]));
+          const float2 g2 = mul2(bf16x2_to_f2_again(gv[i]), bf16x2_to_f2_again(dr[b][w]));
           const float2 r = mul2(fma2(x2, ncoef2, g2), sdx2);
           const __nv_bfloat162 h = __floats2bfloat162_rn(r.x, r.y);
           o[i] = *reinterpret_cast<const uint32_t*>(&h);
