@@ -63,6 +63,7 @@ struct Smem {
   uint64_t mma_done;                             // every MMA of this CTA retired
   uint32_t tmem_base;
   uint32_t failed;
+  uint8_t cstage[kEpiWarps][32 * 64];            // per epilogue warp: 32 rows x 32 bf16 of C
 };
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -278,8 +279,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.acc_empty);  // the MMA thread may overwrite the accumulator
-      const int row = mt * kTileM + quarter * 32 + lane;
-      uint16_t* crow = c + (size_t)row * N + (size_t)nt * kTileN + half * 128;
+      // Each 32-column slice goes through the warp's staging buffer: lane l
+      // writes its row (64 B, 16-byte chunk c at chunk c ^ ((l >> 1) & 3)), then
+      // the warp writes 8 rows x 64 B per store instruction, whole sectors.
+      uint8_t* stg = S.cstage[e];
+      const uint32_t stg_u32 = smem_u32(stg);
+      uint16_t* ctile = c + (size_t)(mt * kTileM + quarter * 32) * N + (size_t)nt * kTileN + half * 128;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t o[16];
@@ -288,9 +293,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[j][2 * i]), __uint_as_float(r[j][2 * i + 1]));
           o[i] = *reinterpret_cast<const uint32_t*>(&h);
         }
+        __syncwarp();                              // the previous slice's reads are done
 #pragma unroll
-        for (int v = 0; v < 4; ++v)
-          *reinterpret_cast<uint4*>(crow + 32 * j + 8 * v) = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t off = (uint32_t)lane * 64u + (uint32_t)((v ^ ((lane >> 1) & 3)) * 16);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg_u32 + off), "r"(o[4 * v]),
+                       "r"(o[4 * v + 1]), "r"(o[4 * v + 2]), "r"(o[4 * v + 3])
+                       : "memory");
+        }
+        __syncwarp();
+#pragma unroll
+        for (int t2 = 0; t2 < 4; ++t2) {
+          const int rr = t2 * 8 + (lane >> 2), cc = lane & 3;
+          const uint4 v4 = lds128(stg_u32 + (uint32_t)rr * 64u + (uint32_t)((cc ^ ((rr >> 1) & 3)) * 16));
+          *reinterpret_cast<uint4*>(ctile + (size_t)rr * N + 32 * j + 8 * cc) = v4;
+        }
       }
     }
   }
