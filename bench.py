@@ -49,6 +49,8 @@ def parse_args():
                     help="also time MXNorm forward over the sweep shapes (16384 x {2048..16384}, p in {1,2,4,inf}, RNE/SR)")
     ap.add_argument("--soak-s", type=float, default=0.5,
                     help="untimed back-to-back steps before timing, so clocks settle under load")
+    ap.add_argument("--profile-only", choices=["fwd", "sr", "mxfp4", "bwd", "gemm"], default=None,
+                    help="run only this kernel, 4 launches on the workload, untimed (for ncu captures)")
     return ap.parse_args()
 
 
@@ -636,8 +638,45 @@ def run_reference(args, rank, world):
     }
 
 
+def run_profile_only(args):
+    """Four untimed launches of one kernel on the workload (the 8192 x 4096
+    batch; the GEMM on the fused QKV weight), for a profiler to capture."""
+    import torch
+    from normalisation_row_bf16_b200 import ops, synthetic
+    w = workload_cfg(args.workload)
+    T, D, p = w["T"], w["D"], w["p"]
+    x = synthetic.activations(T, D, w.get("kind", "outliers"), seed=0, device="cuda")
+    g = synthetic.gamma(D, seed=0, device="cuda")
+    leg = args.profile_only
+    if leg == "bwd":
+        dy = synthetic.upstream_grad(T, D, seed=0, device="cuda")
+        _, _, G = ops.mxnorm_fwd(x, g, p)
+    if leg == "gemm":
+        wt = synthetic.gemm_weight(6144, D, seed=0, device="cuda")
+        aq, a_s, _ = ops.mxnorm_fwd(x, None, p, scale_layout=ops.SCALES_MMA)
+        bq, b_s = ops.fold_weight(wt, g)
+    for i in range(4):
+        if leg == "fwd":
+            ops.mxnorm_fwd(x, g, p)
+        elif leg == "sr":
+            ops.mxnorm_fwd(x, g, p, rounding=ops.SR, seed=i)
+        elif leg == "mxfp4":
+            ops.mxnorm_fwd_ex(x, g, p, elem="e2m1")
+        elif leg == "bwd":
+            ops.mxnorm_bwd(x, dy, g, G)
+        elif leg == "gemm":
+            ops.mxfp8_gemm(aq, a_s, bq, b_s, T, 6144, D)
+    torch.cuda.synchronize()
+    if ops.device_status() != ops.MXN_OK:
+        raise SystemExit("device status not clean")
+    print(json.dumps({"profile_only": leg, "launches": 4}), flush=True)
+
+
 def main():
     args = parse_args()
+    if args.profile_only:
+        run_profile_only(args)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
