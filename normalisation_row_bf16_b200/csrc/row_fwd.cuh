@@ -612,8 +612,8 @@ const void* pick_fwd_shape(int bpt, int tpr) {
     }
   }
   if constexpr (SR) {
-    // stochastic rounding: one block per thread up to 256 blocks per row
-    // (the Philox arithmetic wants warps, not long unrolled bodies)
+    // stochastic rounding: one or two blocks per thread (the Philox
+    // arithmetic wants warps, not long unrolled bodies)
     if (bpt == 1) {
       switch (tpr) {
         case 64: return (const void*)row_fwd_kernel<MODE, 1, 64, SR, HG, ELEM>;
@@ -622,7 +622,14 @@ const void* pick_fwd_shape(int bpt, int tpr) {
         default: return nullptr;
       }
     }
-    if (bpt == 2) return tpr == 256 ? (const void*)row_fwd_kernel<MODE, 2, 256, SR, HG, ELEM> : nullptr;
+    if (bpt == 2) {
+      switch (tpr) {
+        case 64: return (const void*)row_fwd_kernel<MODE, 2, 64, SR, HG, ELEM>;
+        case 128: return (const void*)row_fwd_kernel<MODE, 2, 128, SR, HG, ELEM>;
+        case 256: return (const void*)row_fwd_kernel<MODE, 2, 256, SR, HG, ELEM>;
+        default: return nullptr;
+      }
+    }
   }
   if (bpt != 4) return nullptr;
   switch (tpr) {
