@@ -143,3 +143,44 @@ def test_gemm_argument_checks(L):
     assert f(FAKE, FAKE, MISALIGNED, FAKE, FAKE, 128, 256, 128, None) == ops.MXN_ERR_ARG
     L.mxnorm_debug_fail_next(1)
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 128, None) == ops.MXN_ERR_CUDA
+
+
+def test_codes_bytes(L):
+    assert L.mxnorm_codes_bytes(8192, 4096, 0) == 8192 * 4096
+    assert L.mxnorm_codes_bytes(8192, 4096, 1) == 8192 * 2048
+    assert L.mxnorm_codes_bytes(3, 96, 1) == 3 * 48
+    assert L.mxnorm_codes_bytes(4, 33, 0) == 0
+    assert L.mxnorm_codes_bytes(4, 64, 2) == 0
+    assert L.mxnorm_codes_bytes(-1, 64, 0) == 0
+
+
+def test_variant_entry_points_validate(L):
+    st = None
+    fx = L.mxnorm_fwd_ex
+    # element format and statistic out of range
+    assert fx(FAKE, None, FAKE, FAKE, None, 4, 64, 64, 2.0, 0, 0, 0, 2, 0, st) == ops.MXN_ERR_ARG
+    assert fx(FAKE, None, FAKE, FAKE, None, 4, 64, 64, 2.0, 0, 0, 0, 0, 3, st) == ops.MXN_ERR_ARG
+    # the shared checks still apply
+    assert fx(FAKE, None, FAKE, FAKE, None, 4, 33, 64, 2.0, 0, 0, 0, 1, 0, st) == ops.MXN_ERR_ARG
+    assert fx(FAKE, None, FAKE, FAKE, None, 4, 64, 64, 0.0, 0, 0, 0, 1, 1, st) == ops.MXN_ERR_ARG
+    assert fx(FAKE, None, FAKE, FAKE, None, 0, 64, 64, 2.0, 0, 0, 0, 1, 1, st) == ops.MXN_OK   # empty
+    cx = L.mx_cast_ex
+    assert cx(FAKE, MISALIGNED, FAKE, FAKE, 4, 64, 64, 0, 0, 0, 0, st) == ops.MXN_ERR_ARG
+    assert cx(FAKE, None, FAKE, FAKE, 4, 64, 64, 0, 0, 0, 5, st) == ops.MXN_ERR_ARG
+    assert cx(FAKE, None, None, FAKE, 4, 64, 64, 0, 0, 0, 1, st) == ops.MXN_ERR_ARG
+    fw = L.mxnorm_fold_weight
+    assert fw(FAKE, None, FAKE, FAKE, 4, 64, 64, 0, 1, st) == ops.MXN_ERR_ARG          # nothing to fold
+    assert fw(FAKE, FAKE, FAKE, FAKE, 4, 64, 64, 9, 1, st) == ops.MXN_ERR_ARG
+    assert fw(FAKE, FAKE, FAKE, FAKE, 4, 64, 64, 0, 3, st) == ops.MXN_ERR_ARG
+    assert fw(FAKE, FAKE, FAKE, FAKE, 0, 64, 64, 0, 1, st) == ops.MXN_OK               # empty
+
+
+def test_python_variant_bindings_refuse_cpu_tensors(L):
+    import torch
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ops.mxnorm_fwd_ex(x, elem="e2m1")
+    with pytest.raises(ValueError):
+        ops.mx_cast(x)
+    with pytest.raises(ValueError):
+        ops.fold_weight(x, x[0])
