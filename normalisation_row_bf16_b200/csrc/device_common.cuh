@@ -335,6 +335,21 @@ __device__ __forceinline__ PhiloxKeys philox_keys(uint32_t seed_lo, uint32_t see
   return K;
 }
 
+// Two independent counters in lock-step: the same rounds, interleaved, so each
+// round's multiplies of one stream overlap the other's (two dependency chains).
+__device__ __forceinline__ void philox4x32_10_x2(uint4& a, uint4& b, const PhiloxKeys& K) {
+  constexpr uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t pa0 = (uint64_t)M0 * a.x, pa1 = (uint64_t)M1 * a.z;
+    const uint64_t pb0 = (uint64_t)M0 * b.x, pb1 = (uint64_t)M1 * b.z;
+    a = make_uint4((uint32_t)(pa1 >> 32) ^ a.y ^ K.k0[r], (uint32_t)pa1, (uint32_t)(pa0 >> 32) ^ a.w ^ K.k1[r],
+                   (uint32_t)pa0);
+    b = make_uint4((uint32_t)(pb1 >> 32) ^ b.y ^ K.k0[r], (uint32_t)pb1, (uint32_t)(pb0 >> 32) ^ b.w ^ K.k1[r],
+                   (uint32_t)pb0);
+  }
+}
+
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys& K) {
   constexpr uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
 #pragma unroll

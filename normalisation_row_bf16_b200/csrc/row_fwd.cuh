@@ -277,10 +277,13 @@ __device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a,
     for (int sl = 0; sl < 4; ++sl) {
       const int c = (sl + rot) & 3;
       const uint64_t ctr = (idx0 + (uint64_t)(c * 8)) >> 2;
+      // the slot's two counters (its 8 elements) in one interleaved Philox
+      uint4 rr[2] = {make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), 0u, 0u),
+                     make_uint4((uint32_t)(ctr + 1), (uint32_t)((ctr + 1) >> 32), 0u, 0u)};
+      philox4x32_10_x2(rr[0], rr[1], pk);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const uint64_t cc = ctr + h;
-        const uint4 r = philox4x32_10(make_uint4((uint32_t)cc, (uint32_t)(cc >> 32), 0u, 0u), pk);
+        const uint4 r = rr[h];
         const int i0 = sl * 8 + h * 4;
         const float2 v0 = mul2(make_float2(y[i0], y[i0 + 1]), inv2);
         const float2 v1 = mul2(make_float2(y[i0 + 2], y[i0 + 3]), inv2);
