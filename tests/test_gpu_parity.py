@@ -275,3 +275,30 @@ def test_status_clean_and_empty_input():
     q, s, G = ops.mxnorm_fwd(x)
     assert q.numel() == 0
     assert ops.device_status() == ops.MXN_OK
+
+
+def test_more_than_2_31_elements_sampled_rows():
+    """A 524800 x 4096 tensor (2.15e9 elements, past 32-bit element indices):
+    forward (nearest-even, and stochastic, whose Philox counter is the 64-bit
+    element index / 4) and backward, checked on rows at both ends and around
+    the 2^31-element mark."""
+    T, D = 524800, 4096
+    x = synthetic.activations(T, D, "normal", seed=3, device="cuda")
+    g = synthetic.gamma(D, seed=3, device="cuda")
+    rows = np.array([0, 1, 524287, 524288, T - 2, T - 1])
+    for rounding in (ops.RNE, ops.SR):
+        q, s, G = ops.mxnorm_fwd(x, g, 2.0, rounding=rounding, seed=11)
+        torch.cuda.synchronize()
+        check_mxnorm_fwd(x, g, 2.0, rounding, 11, q, s, G, rows=rows, strict=False)
+        del q, s, G
+        torch.cuda.empty_cache()
+    dy = synthetic.upstream_grad(T, D, seed=3, device="cuda")
+    _, _, G = ops.mxnorm_fwd(x, g, 2.0)
+    dx, dg = ops.mxnorm_bwd(x, dy, g, G)
+    torch.cuda.synchronize()
+    sel = torch.from_numpy(rows).cuda()
+    dx_ref, _ = oracle.mxnorm_bwd(x[sel].cpu(), dy[sel].cpu(), g.cpu(), G[sel].cpu().numpy())
+    assert rel_l2(dx[sel].double().cpu().numpy(), round_bf16(dx_ref)) <= BWD_RTOL_L2
+    assert torch.isfinite(dg.float()).all()
+    del x, dy, dx, G
+    torch.cuda.empty_cache()

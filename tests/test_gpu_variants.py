@@ -210,3 +210,32 @@ def test_fold_weight_requires_gamma_and_checks_format():
     g = _dev(synthetic.gamma(64, seed=0))
     assert L.mxnorm_fold_weight(w.data_ptr(), g.data_ptr(), q.data_ptr(), s.data_ptr(), 4, 64, 64, 7, 0, st) == ops.MXN_ERR_ARG
     assert L.mxnorm_fwd_ex(w.data_ptr(), None, q.data_ptr(), s.data_ptr(), None, 4, 64, 64, 2.0, 0, 0, 0, 0, 5, st) == ops.MXN_ERR_ARG
+
+
+@pytest.mark.parametrize("elem,stat", [("e2m1", "absmax"), ("e4m3", "scale_exp"), ("e2m1", "scale_exp")])
+def test_variants_llama8b_shape_sampled_rows(elem, stat):
+    """The 8192 x 4096 outlier batch with gamma, p = 2: the launches the
+    bench's mxfp4 and scale-reuse legs time, on sampled rows."""
+    w = synthetic.WORKLOADS["llama8b_8192x4096_outliers_p2"]
+    x = synthetic.activations(w["T"], w["D"], w["kind"], seed=0, device="cuda")
+    g = synthetic.gamma(w["D"], seed=0, device="cuda")
+    q, s, G = ops.mxnorm_fwd_ex(x, g, 2.0, elem=elem, stat=stat)
+    torch.cuda.synchronize()
+    rows = np.concatenate([np.arange(0, 8), np.random.default_rng(2).choice(w["T"], 40, replace=False),
+                           np.arange(w["T"] - 8, w["T"])])
+    check_mxnorm_fwd(x, g, 2.0, ops.RNE, 0, q, s, G, rows=rows, strict=False, stat=stat, fmt=elem)
+    for rnd in (ops.SR,):
+        q, s, G = ops.mxnorm_fwd_ex(x, g, 2.0, rounding=rnd, seed=5, elem=elem, stat=stat)
+        torch.cuda.synchronize()
+        check_mxnorm_fwd(x, g, 2.0, rnd, 5, q, s, G, rows=rows[:16], strict=False, stat=stat, fmt=elem)
+
+
+def test_fold_weight_full_qkv_sampled_rows():
+    """The bench's fold_weight launch: the 6144 x 4096 QKV weight times gamma."""
+    w = synthetic.gemm_weight(6144, 4096, seed=0, device="cuda")
+    g = synthetic.gamma(4096, seed=0, device="cuda")
+    q, s = ops.fold_weight(w, g, scale_layout=ops.SCALES_ROWMAJOR)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(4).choice(6144, 64, replace=False)
+    q_ref, s_ref = oracle.mx_cast(w.cpu(), g.cpu(), rows=rows)
+    assert np.array_equal(to_np_u8(q)[rows], q_ref) and np.array_equal(to_np_u8(s)[rows], s_ref)
