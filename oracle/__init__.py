@@ -58,6 +58,7 @@ def _load():
         lib.oracle_e2m1_rne_many.argtypes = [P, i64, P]
         lib.oracle_e2m1_sr_many.argtypes = [P, P, i64, P]
         lib.oracle_mx_exponent_many.argtypes = [P, i64, f64, P]
+        lib.oracle_nvfp4_scale_code_many.argtypes = [P, i64, P]
         lib.oracle_e2m1_value.argtypes = [i32]
         lib.oracle_e2m1_value.restype = f64
         lib.oracle_sr_words.argtypes = [u64, P, i64, P]
@@ -177,7 +178,16 @@ def mx_exponent(a, elem_max: float) -> np.ndarray:
     return out
 
 
-FMT = {"e4m3": 0, "e2m1": 1}
+FMT = {"e4m3": 0, "e2m1": 1, "nvfp4": 2}
+BLOCK = {"e4m3": 32, "e2m1": 32, "nvfp4": 16}
+
+
+def nvfp4_scale_code(a) -> np.ndarray:
+    """E4M3 code of the smallest E4M3 value s with |a| <= 6 s (NVFP4 block scale)."""
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    out = np.empty(a.shape, np.int32)
+    _load().oracle_nvfp4_scale_code_many(_ptr(a), a.size, _ptr(out))
+    return out
 STAT = {"absmax": 0, "scale_exp": 1}
 
 
@@ -231,15 +241,16 @@ def mxnorm_fwd(x, gamma=None, p: float = 2.0, rows=None, G_in=None, rounding: in
 def mxnorm_fwd_ex(x, gamma=None, p: float = 2.0, rows=None, G_in=None, rounding: int = 0,
                   seed: int = 0, stat: str = "absmax", fmt: str = "e4m3", nthreads: int = 0):
     """MXNorm forward with a choice of block statistic ("absmax", or "scale_exp":
-    the block's power-of-two scale) and element format ("e4m3", or "e2m1" with
-    two codes per byte, q uint8 [n, D/2]).  Returns (q, scales, G)."""
+    the block's scale) and element format ("e4m3"; "e2m1" with two codes per
+    byte, q uint8 [n, D/2]; "nvfp4": E2M1 codes with one E4M3 scale per 16,
+    scales uint8 [n, D/16]).  Returns (q, scales, G)."""
     xu = _u16(x)
     T, D = xu.shape
     g = _u16(gamma)
     r, n = _rows(rows, T)
     Gi = None if G_in is None else np.ascontiguousarray(np.asarray(G_in, np.float32).reshape(n))
-    q = np.empty((n, D // 2 if fmt == "e2m1" else D), np.uint8)
-    s = np.empty((n, D // 32), np.uint8)
+    q = np.empty((n, D if fmt == "e4m3" else D // 2), np.uint8)
+    s = np.empty((n, D // BLOCK[fmt]), np.uint8)
     G = np.empty(n, np.float32)
     rc = _load().oracle_mxnorm_fwd_ex(_ptr(xu), D, _ptr(g), n, _ptr(r), D, float(p), _ptr(Gi),
                                       _ptr(q), _ptr(s), _ptr(G), int(rounding),
@@ -257,8 +268,8 @@ def mx_cast(x, gamma=None, rows=None, rounding: int = 0, seed: int = 0, fmt: str
     T, D = xu.shape
     g = _u16(gamma)
     r, n = _rows(rows, T)
-    q = np.empty((n, D // 2 if fmt == "e2m1" else D), np.uint8)
-    s = np.empty((n, D // 32), np.uint8)
+    q = np.empty((n, D if fmt == "e4m3" else D // 2), np.uint8)
+    s = np.empty((n, D // BLOCK[fmt]), np.uint8)
     rc = _load().oracle_mx_cast_ex(_ptr(xu), D, _ptr(g), n, _ptr(r), D, _ptr(q), _ptr(s),
                                    int(rounding), ctypes.c_uint64(seed), FMT[fmt], int(nthreads))
     if rc != 0:

@@ -40,6 +40,14 @@
  *  [SE]  Scale reuse (the MXNorm title: reusing the block scales): the block
  *        statistic m_k replaced by the block's own power-of-two scale 2^e_k,
  *        e_k the [RC] exponent of m_k.
+ *  [NV]  NVFP4, the FP4 format the MXNorm summary (section 3) reports its
+ *        layer speedup with; the pages name it without defining it.  Reading
+ *        adopted: E2M1 elements [F4] in blocks of 16, each block with a
+ *        positive E4M3 scale [F8], the smallest E4M3 value s with
+ *        amax <= 6 s (rounded up, as [RC]), and no tensor-wide scale (MXNorm
+ *        already bounds |y| by K^(1/p) max|gamma|, so the scales stay inside
+ *        E4M3's range); codes E2M1(fl32(y * fl32(1/s))).  The MXNorm statistic
+ *        then runs over the 16-element blocks.
  *
  * Precision: statistics (G, RMS, backward sums) in long double / double.
  * Where floating point decides an integer code, the oracle takes that decision
@@ -61,6 +69,8 @@
 #define E2M1_MAX 6.0             /* [F4] */
 #define ORACLE_FMT_E4M3 0
 #define ORACLE_FMT_E2M1 1
+#define ORACLE_FMT_NVFP4 2
+#define NVFP4_BLOCK 16           /* [NV] */
 
 /* ---------------------------------------------------------------- helpers */
 
@@ -346,6 +356,55 @@ static void mx_quantise_row(const float *y, int64_t D, uint8_t *q, uint8_t *scal
     }
 }
 
+/* The NVFP4 block scale [NV]: the E4M3 code of the smallest E4M3 value s with
+   a <= 6 * s (6 * s is exact in double); 0x7E (448) if none, 0 for a = 0. */
+int oracle_nvfp4_scale_code(double a)
+{
+    for (int c = 0; c <= 0x7E; ++c)
+        if (a <= 6.0 * oracle_e4m3_value(c)) return c;
+    return 0x7E;
+}
+
+/* Quantise one row y[0..D) to NVFP4 [NV]: per block of 16, the E4M3 scale
+   code (scales[k]) and the E2M1 codes of fl32(y * fl32(1/s)), two per byte,
+   even column in the low nibble.  A zero scale (an all-zero block) gives
+   zero codes; a block holding an infinity or a NaN gets the E4M3 NaN scale
+   0x7F and element code 0x7. */
+static void nvfp4_quantise_row(const float *y, int64_t D, uint8_t *q, uint8_t *scales,
+                               int rounding, uint64_t seed, uint64_t row)
+{
+    int64_t K = D / NVFP4_BLOCK;
+    memset(q, 0, (size_t)(D / 2));
+    for (int64_t k = 0; k < K; ++k) {
+        const float *yb = y + k * NVFP4_BLOCK;
+        double a = 0.0;
+        int nonfinite = 0;
+        for (int i = 0; i < NVFP4_BLOCK; ++i) {
+            double v = fabs((double)yb[i]);
+            if (!(v <= DBL_MAX)) nonfinite = 1;
+            else if (v > a) a = v;
+        }
+        int sc = nonfinite ? 0x7F : oracle_nvfp4_scale_code(a);
+        scales[k] = (uint8_t)sc;
+        float sval = (float)oracle_e4m3_value(sc & 0x7F);
+        float inv = (sc == 0 || nonfinite) ? 0.0f : 1.0f / sval;   /* fl32(1/s) */
+        for (int i = 0; i < NVFP4_BLOCK; ++i) {
+            int64_t col = k * NVFP4_BLOCK + i;
+            uint8_t c;
+            if (nonfinite) {
+                c = 0x7;
+            } else if (sc == 0) {
+                c = 0;
+            } else {
+                float v = yb[i] * inv;
+                c = rounding ? oracle_e2m1_sr(v, sr_word(seed, row * (uint64_t)D + (uint64_t)col))
+                             : oracle_e2m1_rne(v);
+            }
+            q[col / 2] |= (uint8_t)(c << (4 * (col & 1)));
+        }
+    }
+}
+
 static const uint16_t *row_ptr(const uint16_t *base, int64_t ld, int64_t r) { return base + r * ld; }
 
 static int64_t pick_row(const int64_t *row_ids, int64_t i) { return row_ids ? row_ids[i] : i; }
@@ -371,9 +430,10 @@ int oracle_mxnorm_fwd_ex(const uint16_t *x, int64_t ld_x, const uint16_t *gamma,
                          int rounding, uint64_t seed, int stat, int fmt, int nthreads)
 {
     if (D <= 0 || D % ORACLE_BLOCK != 0 || !(p > 0.0)) return -1;
-    if (fmt != ORACLE_FMT_E4M3 && fmt != ORACLE_FMT_E2M1) return -1;
-    int64_t K = D / ORACLE_BLOCK;
-    const int64_t qrow = (fmt == ORACLE_FMT_E2M1) ? D / 2 : D;
+    if (fmt != ORACLE_FMT_E4M3 && fmt != ORACLE_FMT_E2M1 && fmt != ORACLE_FMT_NVFP4) return -1;
+    const int B = (fmt == ORACLE_FMT_NVFP4) ? NVFP4_BLOCK : ORACLE_BLOCK;   /* statistic blocks */
+    int64_t K = D / B;
+    const int64_t qrow = (fmt == ORACLE_FMT_E4M3) ? D : D / 2;
     const double elem_max = (fmt == ORACLE_FMT_E2M1) ? E2M1_MAX : E4M3_MAX;
 #ifdef _OPENMP
     if (nthreads <= 0) nthreads = omp_get_max_threads();
@@ -386,11 +446,14 @@ int oracle_mxnorm_fwd_ex(const uint16_t *x, int64_t ld_x, const uint16_t *gamma,
         float y[D];
         for (int64_t k = 0; k < K; ++k) {
             double mk = 0.0;
-            for (int j = 0; j < ORACLE_BLOCK; ++j) {
-                double v = fabs((double)bf16_to_f32(xr[k * ORACLE_BLOCK + j]));
+            for (int j = 0; j < B; ++j) {
+                double v = fabs((double)bf16_to_f32(xr[k * B + j]));
                 if (isnan(v) || v > mk) mk = v;   /* a NaN, once seen, stays the max */
             }
-            if (stat == 1 && mk <= DBL_MAX) mk = ldexp(1.0, oracle_mx_exponent(mk, elem_max));
+            if (stat == 1 && mk <= DBL_MAX) {
+                if (fmt == ORACLE_FMT_NVFP4) mk = oracle_e4m3_value(oracle_nvfp4_scale_code(mk));
+                else mk = ldexp(1.0, oracle_mx_exponent(mk, elem_max));
+            }
             m[k] = mk;
         }
         float G_ref = (float)pmean(m, K, p);
@@ -401,7 +464,10 @@ int oracle_mxnorm_fwd_ex(const uint16_t *x, int64_t ld_x, const uint16_t *gamma,
             float t = bf16_to_f32(xr[j]) * s;
             y[j] = gamma ? t * bf16_to_f32(gamma[j]) : t;
         }
-        mx_quantise_row(y, D, q + i * qrow, scales + i * K, rounding, seed, (uint64_t)r, fmt);
+        if (fmt == ORACLE_FMT_NVFP4)
+            nvfp4_quantise_row(y, D, q + i * qrow, scales + i * K, rounding, seed, (uint64_t)r);
+        else
+            mx_quantise_row(y, D, q + i * qrow, scales + i * K, rounding, seed, (uint64_t)r, fmt);
     }
     (void)nthreads;
     return 0;
@@ -427,9 +493,9 @@ int oracle_mx_cast_ex(const uint16_t *x, int64_t ld_x, const uint16_t *gamma, in
                       int rounding, uint64_t seed, int fmt, int nthreads)
 {
     if (D <= 0 || D % ORACLE_BLOCK != 0) return -1;
-    if (fmt != ORACLE_FMT_E4M3 && fmt != ORACLE_FMT_E2M1) return -1;
-    int64_t K = D / ORACLE_BLOCK;
-    const int64_t qrow = (fmt == ORACLE_FMT_E2M1) ? D / 2 : D;
+    if (fmt != ORACLE_FMT_E4M3 && fmt != ORACLE_FMT_E2M1 && fmt != ORACLE_FMT_NVFP4) return -1;
+    int64_t K = D / ((fmt == ORACLE_FMT_NVFP4) ? NVFP4_BLOCK : ORACLE_BLOCK);
+    const int64_t qrow = (fmt == ORACLE_FMT_E4M3) ? D : D / 2;
 #ifdef _OPENMP
     if (nthreads <= 0) nthreads = omp_get_max_threads();
 #pragma omp parallel for schedule(dynamic, 4) num_threads(nthreads)
@@ -442,7 +508,10 @@ int oracle_mx_cast_ex(const uint16_t *x, int64_t ld_x, const uint16_t *gamma, in
             float t = bf16_to_f32(xr[j]);
             y[j] = gamma ? t * bf16_to_f32(gamma[j]) : t;
         }
-        mx_quantise_row(y, D, q + i * qrow, scales + i * K, rounding, seed, (uint64_t)r, fmt);
+        if (fmt == ORACLE_FMT_NVFP4)
+            nvfp4_quantise_row(y, D, q + i * qrow, scales + i * K, rounding, seed, (uint64_t)r);
+        else
+            mx_quantise_row(y, D, q + i * qrow, scales + i * K, rounding, seed, (uint64_t)r, fmt);
     }
     (void)nthreads;
     return 0;
@@ -596,6 +665,11 @@ void oracle_e2m1_rne_many(const float *v, int64_t n, uint8_t *out)
 void oracle_e2m1_sr_many(const float *v, const uint32_t *r, int64_t n, uint8_t *out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_e2m1_sr(v[i], r[i]);
+}
+
+void oracle_nvfp4_scale_code_many(const float *a, int64_t n, int32_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_nvfp4_scale_code(fabs((double)a[i]));
 }
 
 void oracle_mx_exponent_many(const float *a, int64_t n, double elem_max, int32_t *out)

@@ -1,4 +1,4 @@
-"""Pins for the oracle's MXFP4 element format, scale-reuse statistic and gain cast.
+"""Pins for the oracle's MXFP4 and NVFP4 formats, scale-reuse statistic and gain cast.
 
 Each check compares the oracle with something other than itself:
 
@@ -17,6 +17,11 @@ Each check compares the oracle with something other than itself:
 * Gain cast (MXNormLinear's folded weight, MXNorm summary section 2.3): gamma
   of ones gives the plain cast, power-of-two gains only move the scales, and a
   float32 recomputation with torch's float8 cast.
+* NVFP4 (E2M1 in blocks of 16 with E4M3 scales, read as having no tensor-wide
+  scale): the scale code against a search of torch's float8_e4m3fn grid, whole
+  rows against a python recomputation (scipy p-mean over the 16-element block
+  maxima, grid search for the scales, ml_dtypes for the codes), 2^t scaling,
+  zero blocks, the gain cast and the scale-reuse statistic.
 """
 import math
 
@@ -268,3 +273,88 @@ def test_gain_cast_pins():
         enc = lambda v: torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
         sw, cw = _python_mx_row(y, 448.0, enc)
         assert np.array_equal(s3[r], sw) and np.array_equal(q3[r], cw)
+
+
+# ---------------------------------------------------------------- NVFP4
+
+E4M3_POS = torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+
+
+def _brute_nvfp4_scale_code(a):
+    ok = np.nonzero(6.0 * E4M3_POS >= a)[0]
+    return int(ok[0]) if ok.size else 0x7E
+
+
+def test_nvfp4_scale_code_vs_e4m3_grid():
+    rng = np.random.default_rng(7)
+    a = np.concatenate([[0.0, 1e-6, 6 * 2.0 ** -9, 6 * 2.0 ** -9 * 1.0001, 6.0, 6.0001, 2688.0, 2689.0, 1e30],
+                        np.exp(rng.uniform(np.log(1e-5), np.log(3000.0), 4000))]).astype(np.float32)
+    got = oracle.nvfp4_scale_code(a)
+    want = np.array([_brute_nvfp4_scale_code(float(v)) for v in a])
+    assert np.array_equal(got, want)
+    # every grid value times 6 is its own threshold: a = 6 s gives s exactly
+    for c in range(1, 127):
+        assert oracle.nvfp4_scale_code([np.float32(6.0 * E4M3_POS[c])])[0] == c
+
+
+def _python_nvfp4_row(y):
+    scales, codes = [], []
+    for k in range(y.size // 16):
+        blk = y[16 * k:16 * (k + 1)]
+        a = float(np.max(np.abs(blk.astype(np.float64))))
+        c = _brute_nvfp4_scale_code(a)
+        scales.append(c)
+        if c == 0:
+            codes.append(np.zeros(16, np.uint8))
+            continue
+        inv = np.float32(1.0) / np.float32(E4M3_POS[c])
+        codes.append(_ml_e2m1_codes((blk * inv).astype(np.float32)))
+    return np.array(scales, np.uint8), _pack_e2m1(np.concatenate(codes))
+
+
+@pytest.mark.parametrize("p", [1.0, 2.0, 4.0, math.inf])
+def test_nvfp4_rows_vs_python(p):
+    T, D = 5, 256
+    x = synthetic.activations(T, D, "outliers", seed=12)
+    g = synthetic.gamma(D, seed=12)
+    q, s, G = oracle.mxnorm_fwd_ex(x, g, p, fmt="nvfp4")
+    assert q.shape == (T, D // 2) and s.shape == (T, D // 16)
+    xf, gf = x.float().numpy(), g.float().numpy()
+    for t in range(T):
+        m = np.abs(xf[t].reshape(-1, 16).astype(np.float64)).max(1)       # 16-element blocks
+        Gw = np.float32(m.max() if math.isinf(p) else scipy.stats.pmean(m, p))
+        assert abs(float(G[t]) - float(Gw)) <= 1e-6 * float(Gw)
+        y = ((xf[t] * (np.float32(1.0) / G[t])).astype(np.float32) * gf).astype(np.float32)
+        sw, qw = _python_nvfp4_row(y)
+        assert np.array_equal(s[t], sw) and np.array_equal(q[t], qw)
+
+
+def test_nvfp4_invariants_and_zero_blocks():
+    x = synthetic.activations(4, 128, "student_t", seed=2)
+    q0, s0, G0 = oracle.mxnorm_fwd_ex(x, None, 2.0, fmt="nvfp4")
+    for t in (-5, 7):
+        q1, s1, G1 = oracle.mxnorm_fwd_ex((x.float() * 2.0 ** t).to(torch.bfloat16), None, 2.0, fmt="nvfp4")
+        assert np.array_equal(q1, q0) and np.array_equal(s1, s0)
+        assert np.array_equal(G1, G0 * np.float32(2.0 ** t))
+    z = x.clone()
+    z[1, 16:32] = 0
+    q, s, _ = oracle.mxnorm_fwd_ex(z, None, 2.0, fmt="nvfp4")
+    assert s[1, 1] == 0 and np.all(q[1, 8:16] == 0)
+    # the gain cast in NVFP4 is the python row on fl32(x * gain)
+    g = synthetic.gamma(128, seed=4)
+    qc, sc = oracle.mx_cast(x, g, fmt="nvfp4")
+    for r in range(4):
+        y = (x.float().numpy()[r] * g.float().numpy()).astype(np.float32)
+        sw, qw = _python_nvfp4_row(y)
+        assert np.array_equal(sc[r], sw) and np.array_equal(qc[r], qw)
+
+
+def test_nvfp4_scale_reuse_statistic():
+    x = synthetic.activations(3, 256, "outliers", seed=9)
+    _, _, G = oracle.mxnorm_fwd_ex(x, None, 2.0, stat="scale_exp", fmt="nvfp4")
+    xf = x.float().numpy().astype(np.float64)
+    for t in range(3):
+        m = np.abs(xf[t]).reshape(-1, 16).max(1)
+        sv = np.array([E4M3_POS[_brute_nvfp4_scale_code(a)] for a in m])
+        want = scipy.stats.pmean(sv, 2.0)
+        assert abs(float(G[t]) - want) <= 1e-6 * want
