@@ -49,7 +49,7 @@ def parse_args():
                     help="also time MXNorm forward over the sweep shapes (16384 x {2048..16384}, p in {1,2,4,inf}, RNE/SR)")
     ap.add_argument("--soak-s", type=float, default=0.5,
                     help="untimed back-to-back steps before timing, so clocks settle under load")
-    ap.add_argument("--profile-only", choices=["fwd", "sr", "mxfp4", "bwd", "gemm"], default=None,
+    ap.add_argument("--profile-only", choices=["fwd", "sr", "mxfp4", "nvfp4", "bwd", "gemm"], default=None,
                     help="run only this kernel, 4 launches on the workload, untimed (for ncu captures)")
     return ap.parse_args()
 
@@ -389,6 +389,15 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
                                                                  G=outs4[i % n_sets][2]),
                                      fp4_bytes(T, D), "row_fwd_kernel<MXNorm, E2M1>")
     del outs4
+    outsn = [(torch.empty(T, D // 2, dtype=torch.uint8, device=dev),
+              torch.empty(T, D // 16, dtype=torch.uint8, device=dev),
+              torch.empty(T, dtype=torch.float32, device=dev)) for _ in range(n_sets)]
+    out["nvfp4_fwd"] = run_graph_leg(args, world, dev, barrier,
+                                     lambda i: ops.mxnorm_fwd_ex(xs[i % n_sets], g, p, elem="nvfp4",
+                                                                 q=outsn[i % n_sets][0], scales=outsn[i % n_sets][1],
+                                                                 G=outsn[i % n_sets][2]),
+                                     nvfp4_bytes(T, D), "row_fwd_kernel<MXNorm, NVFP4>")
+    del outsn
     outs = [(torch.empty(T, D, dtype=torch.uint8, device=dev), torch.empty(T, D // 32, dtype=torch.uint8, device=dev),
              torch.empty(T, dtype=torch.float32, device=dev)) for _ in range(n_sets)]
     out["scale_reuse_fwd"] = run_graph_leg(args, world, dev, barrier,
@@ -536,6 +545,11 @@ def run_gemm_leg(args, w, rank, world, dev, barrier):
             "kernel": "gemm_mxfp8_kernel (tcgen05 mxf8f6f4 block_scale, 128x256 tiles)"}
 
 
+def nvfp4_bytes(T, D):
+    # read x (2 B/elem), write E2M1 codes (1/2 B/elem) and E4M3 scales (1 per 16); gamma, G
+    return int(T * D * 2 + T * D // 2 + T * (D // 16) + 2 * D + 4 * T)
+
+
 def fp4_bytes(T, D):
     # read x (2 B/elem), write E2M1 codes (1/2 B/elem) and scales (1/32); gamma, G
     return int(T * D * 2 + T * D // 2 + T * (D // 32) + 2 * D + 4 * T)
@@ -662,6 +676,8 @@ def run_profile_only(args):
             ops.mxnorm_fwd(x, g, p, rounding=ops.SR, seed=i)
         elif leg == "mxfp4":
             ops.mxnorm_fwd_ex(x, g, p, elem="e2m1")
+        elif leg == "nvfp4":
+            ops.mxnorm_fwd_ex(x, g, p, elem="nvfp4")
         elif leg == "bwd":
             ops.mxnorm_bwd(x, dy, g, G)
         elif leg == "gemm":

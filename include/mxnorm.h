@@ -98,7 +98,18 @@ enum mxn_elem_format {
        in bits 0..3: codes [T, D / 2].  Scale rule as for E4M3 with 6 in
        place of 448; nearest-even saturates to +-6; a block holding NaN or
        infinity gets scale 0xFF and element code 0x7. */
-    MXN_ELEM_E2M1 = 1
+    MXN_ELEM_E2M1 = 1,
+    /* NVFP4 (the FP4 format the MXNorm summary's section 3 quotes its layer
+       speedup with; the pages do not define it): E2M1 codes packed as for
+       MXN_ELEM_E2M1, codes [T, D / 2], in blocks of 16 elements, each with an
+       E4M3 scale s, the smallest E4M3 value with amax <= 6 * s; codes are
+       E2M1(fl32(y * fl32(1 / s))).  No tensor-wide scale: MXNorm's output is
+       bounded by K^(1/p) * max|gamma|, which keeps every s inside E4M3.
+       Scales: uint8 [T, D / 16] row-major (MXN_SCALES_ROWMAJOR only).  An
+       all-zero block gets scale 0 and codes 0; a block holding NaN or
+       infinity scale 0x7F and codes 0x7.  MXNorm's statistic runs over the
+       16-element blocks (K = D / 16). */
+    MXN_ELEM_NVFP4 = 2
 };
 
 /* Block statistic of the MXNorm p-mean. */
@@ -106,8 +117,8 @@ enum mxn_statistic {
     MXN_STAT_ABSMAX = 0,     /* m_k = block absmax of x (section 2.1) */
     /* Scale reuse (the MXNorm title: reusing the MX block scales): m_k is
        replaced by 2^e_k, e_k the scale exponent of block k of x by the rule
-       above for the element format (a zero block gives 2^-127); infinities
-       and NaN pass through. */
+       above for the element format (a zero block gives 2^-127); for NVFP4 by
+       the block's E4M3 scale value; infinities and NaN pass through. */
     MXN_STAT_SCALE_EXP = 1
 };
 

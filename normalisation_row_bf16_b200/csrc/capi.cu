@@ -183,6 +183,7 @@ int check_opt(const void* p, const char* name) {
 }
 
 const void* fwd_kernel(int mode, bool sr, bool has_gamma, int elem, int bpt, int tpr) {
+  if (elem == kElemNVFP4) return fwd_kernel_nvfp4(mode, bpt, tpr, sr, has_gamma);
   if (elem == kElemE2M1) {
     switch (mode) {
       case kModeMXNorm:
@@ -315,7 +316,7 @@ int launch_fwd(int mode, bool sr, const FwdArgs& A, int64_t T, int D, int64_t ld
   if (rc) return rc;
   FwdArgs a = A;
   a.status = dev.status;
-  a.inv_K = 1.0f / (float)(D / kBlock);
+  a.inv_K = 1.0f / (float)(A.elem == kElemNVFP4 ? D / 16 : D / kBlock);   // statistic blocks per row
   void* argv[] = {&a, &P.C};
   return launch_pdl(P.kernel, P.grid, P.threads, P.smem, argv, stream, "row_fwd_kernel launch");
 }
@@ -490,12 +491,15 @@ static int fwd_like(int mode, const void* x, const void* gamma, void* q, void* s
     return fail(MXN_ERR_ARG, "rounding = %d", rounding);
   if (scale_layout != MXN_SCALES_ROWMAJOR && scale_layout != MXN_SCALES_MMA)
     return fail(MXN_ERR_ARG, "scale_layout = %d", scale_layout);
-  if (elem != MXN_ELEM_E4M3 && elem != MXN_ELEM_E2M1) return fail(MXN_ERR_ARG, "elem_format = %d", elem);
+  if (elem != MXN_ELEM_E4M3 && elem != MXN_ELEM_E2M1 && elem != MXN_ELEM_NVFP4)
+    return fail(MXN_ERR_ARG, "elem_format = %d", elem);
+  if (elem == MXN_ELEM_NVFP4 && scale_layout != MXN_SCALES_ROWMAJOR)
+    return fail(MXN_ERR_UNSUPPORTED, "NVFP4 scales are row-major only");
   if (stat != MXN_STAT_ABSMAX && stat != MXN_STAT_SCALE_EXP) return fail(MXN_ERR_ARG, "statistic = %d", stat);
   if ((rc = injected())) return rc;
   if (T == 0) return MXN_OK;
   FwdArgs A{};
-  A.elem = elem == MXN_ELEM_E2M1 ? kElemE2M1 : kElemE4M3;
+  A.elem = elem == MXN_ELEM_NVFP4 ? kElemNVFP4 : (elem == MXN_ELEM_E2M1 ? kElemE2M1 : kElemE4M3);
   A.stat_exp = stat == MXN_STAT_SCALE_EXP;
   A.x = static_cast<const uint16_t*>(x);
   A.gamma = static_cast<const uint16_t*>(gamma);
@@ -551,7 +555,7 @@ int mxnorm_fold_weight(const void* w, const void* gamma, void* q, void* scales, 
 size_t mxnorm_codes_bytes(int64_t T, int64_t D, int elem_format) {
   if (T < 0 || D <= 0 || D % kBlock != 0) return 0;
   if (elem_format == MXN_ELEM_E4M3) return (size_t)(T * D);
-  if (elem_format == MXN_ELEM_E2M1) return (size_t)(T * (D / 2));
+  if (elem_format == MXN_ELEM_E2M1 || elem_format == MXN_ELEM_NVFP4) return (size_t)(T * (D / 2));
   return 0;
 }
 

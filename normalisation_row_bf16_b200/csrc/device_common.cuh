@@ -6,6 +6,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -293,6 +294,32 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4_rn(float a, float b, float c, flo
       : "=r"(r)
       : "f"(a), "f"(b), "f"(c), "f"(d));
   return r;
+}
+
+// ------------------------------------------------------------------ NVFP4 scale
+
+// fp32 value of a non-negative E4M3 code (0..0x7E), by the hardware decoder.
+__device__ __forceinline__ float e4m3_to_float(uint32_t c) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
+      : "=r"(h2)
+      : "r"(c));
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// The NVFP4 block scale: the E4M3 code of the smallest E4M3 value s with
+// a <= 6 s (a >= 0 finite), 0x7E when even 448 is too small.  The estimate
+// E4M3(a / 6) is within one code of it (E4M3's relative spacing is >= 1/16,
+// the estimate's error ~1e-7), and 6 s is exact in fp32, so one comparison
+// each way settles it.
+__device__ __forceinline__ uint32_t nvfp4_scale_code(float a) {
+  if (a > 2688.0f) return 0x7Eu;
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(a * (1.0f / 6.0f)));
+  uint32_t c = r & 0xFFu;
+  if (6.0f * e4m3_to_float(c) < a) c += 1;
+  else if (c > 0 && 6.0f * e4m3_to_float(c - 1) >= a) c -= 1;
+  return c > 0x7Eu ? 0x7Eu : c;
 }
 
 // ------------------------------------------------------------------ E2M1 cast

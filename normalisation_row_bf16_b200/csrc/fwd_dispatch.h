@@ -13,5 +13,7 @@ const void* fwd_kernel_rmsnorm(int bpt, int tpr, bool has_gamma);
 const void* fwd_kernel_mxnorm_fp4_rne(int bpt, int tpr, bool has_gamma);
 const void* fwd_kernel_mxnorm_fp4_sr(int bpt, int tpr, bool has_gamma);
 const void* fwd_kernel_cast_fp4(int bpt, int tpr, bool sr, bool has_gamma);
+// NVFP4 codes (E2M1, E4M3 scale per 16): MXNorm and MXCast.
+const void* fwd_kernel_nvfp4(int mode, int bpt, int tpr, bool sr, bool has_gamma);
 
 }  // namespace mxn

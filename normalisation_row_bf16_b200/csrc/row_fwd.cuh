@@ -37,9 +37,10 @@
 namespace mxn {
 
 enum RowMode { kModeMXNorm = 0, kModeCast = 1, kModeRMSNorm = 2 };
-// Element formats of the MX codes: E4M3 (MXFP8, a byte per code) and E2M1
-// (MXFP4, two codes per byte, the even column in the low nibble).
-enum ElemFormat { kElemE4M3 = 0, kElemE2M1 = 1 };
+// Element formats of the codes: E4M3 (MXFP8, a byte per code), E2M1 (MXFP4,
+// two codes per byte, the even column in the low nibble), and NVFP4 (E2M1
+// codes packed the same way, one E4M3 scale per 16 elements).
+enum ElemFormat { kElemE4M3 = 0, kElemE2M1 = 1, kElemNVFP4 = 2 };
 enum PMode { kP1 = 1, kP2 = 2, kP4 = 4, kPInf = 0, kPGeneral = 3 };
 
 // Threads per CTA the register budget is sized for: a thread holding 4 blocks
@@ -310,6 +311,79 @@ __device__ __forceinline__ void store_codes(uint8_t* qp, const uint32_t (&qw)[8]
                  : "memory");
 }
 
+// bf16 magnitude bits of the two 16-element halves of a block held in slot
+// order (slot j holds chunk (j + rot) & 3; chunks 0-1 form half 0).  NaN
+// magnitudes compare above infinity, so a NaN stays the maximum.
+__device__ __forceinline__ void half_absmax_bits(const uint32_t (&w)[16], int rot, uint32_t& h0, uint32_t& h1) {
+  uint32_t sm[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t a = bf16x2_maxabs(bf16x2_maxabs(w[4 * j], w[4 * j + 1]), bf16x2_maxabs(w[4 * j + 2], w[4 * j + 3]));
+    sm[j] = max(a & 0x7FFFu, (a >> 16) & 0x7FFFu);
+  }
+  const uint32_t p01 = max(sm[0], sm[1]), p12 = max(sm[1], sm[2]), p23 = max(sm[2], sm[3]), p30 = max(sm[3], sm[0]);
+  h0 = rot == 0 ? p01 : (rot == 1 ? p30 : (rot == 2 ? p23 : p12));
+  h1 = rot == 0 ? p23 : (rot == 1 ? p12 : (rot == 2 ? p01 : p30));
+}
+
+// NVFP4 quantisation of one 32-element block (two 16-element NVFP4 blocks)
+// held in slot order: per half, the E4M3 scale code (nvfp4_scale_code of the
+// half's absmax, 0x7F for a half holding NaN or infinity), then the E2M1
+// codes of fl32(y * fl32(1/s)); a zero scale gives zero codes, a NaN half
+// codes 0x7.  Returns the two scale codes (half 0 in bits 0..7).
+template <bool SR>
+__device__ __forceinline__ uint32_t quantise_nvfp4(const float (&y)[32], int rot, uint64_t idx0,
+                                                   const PhiloxKeys& pk, uint32_t (&qw)[8]) {
+  float sm[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float m0 = max3_abs_nan(0.0f, y[8 * j], y[8 * j + 1]);
+    float m1 = max3_abs_nan(0.0f, y[8 * j + 2], y[8 * j + 3]);
+    m0 = max3_abs_nan(m0, y[8 * j + 4], y[8 * j + 5]);
+    m1 = max3_abs_nan(m1, y[8 * j + 6], y[8 * j + 7]);
+    sm[j] = max3_abs_nan(m0, m1, 0.0f);
+  }
+  const float p01 = max3_abs_nan(sm[0], sm[1], 0.0f), p12 = max3_abs_nan(sm[1], sm[2], 0.0f);
+  const float p23 = max3_abs_nan(sm[2], sm[3], 0.0f), p30 = max3_abs_nan(sm[3], sm[0], 0.0f);
+  const float ah0 = rot == 0 ? p01 : (rot == 1 ? p30 : (rot == 2 ? p23 : p12));
+  const float ah1 = rot == 0 ? p23 : (rot == 1 ? p12 : (rot == 2 ? p01 : p30));
+  const bool bad0 = !(ah0 <= 3.402823466e38f), bad1 = !(ah1 <= 3.402823466e38f);   // NaN or infinity
+  const uint32_t c0 = bad0 ? 0x7Fu : nvfp4_scale_code(ah0), c1 = bad1 ? 0x7Fu : nvfp4_scale_code(ah1);
+  const float inv0 = (bad0 || c0 == 0) ? 0.0f : __frcp_rn(e4m3_to_float(c0));
+  const float inv1 = (bad1 || c1 == 0) ? 0.0f : __frcp_rn(e4m3_to_float(c1));
+#pragma unroll
+  for (int sl = 0; sl < 4; ++sl) {
+    const bool h1 = (((sl + rot) & 3) >> 1) != 0;
+    const float inv = h1 ? inv1 : inv0;
+    const bool bad = h1 ? bad1 : bad0;
+    const bool zero = (h1 ? c1 : c0) == 0;
+    const float2 inv2 = make_float2(inv, inv);
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 t = mul2(make_float2(y[8 * sl + 2 * i], y[8 * sl + 2 * i + 1]), inv2);
+      v[2 * i] = t.x;
+      v[2 * i + 1] = t.y;
+    }
+    if constexpr (SR) {
+      const int c = (sl + rot) & 3;
+      const uint64_t ctr = (idx0 + (uint64_t)(c * 8)) >> 2;
+      uint4 rr[2] = {make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), 0u, 0u),
+                     make_uint4((uint32_t)(ctr + 1), (uint32_t)((ctr + 1) >> 32), 0u, 0u)};
+      philox4x32_10_x2(rr[0], rr[1], pk);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        v[4 * h] = sr_e2m1_grid(v[4 * h], rr[h].x);
+        v[4 * h + 1] = sr_e2m1_grid(v[4 * h + 1], rr[h].y);
+        v[4 * h + 2] = sr_e2m1_grid(v[4 * h + 2], rr[h].z);
+        v[4 * h + 3] = sr_e2m1_grid(v[4 * h + 3], rr[h].w);
+      }
+    }
+    qw[sl] = bad ? 0x77777777u : (zero ? 0u : cvt_e2m1x8_rn(v));
+  }
+  return c0 | (c1 << 8);
+}
+
 // E2M1 codes of a block (16 bytes): slot j's word goes to bytes
 // 4 * ((j + rot) & 3) .. + 3.
 __device__ __forceinline__ void store_codes_e2m1(uint8_t* qp, const uint32_t (&qw)[8], int rot) {
@@ -532,10 +606,28 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
       // ------------------------------------------------- MXNorm / MXCast
       float sc = 1.0f;
       if constexpr (MODE == kModeMXNorm) {
-        uint32_t mst[BPT];
+        float G;
+        if constexpr (ELEM == kElemNVFP4) {
+          // the statistic runs over the 16-element blocks; its scale-reuse form
+          // uses the blocks' E4M3 scale values (exact in bf16)
+          uint32_t mst[2 * BPT];
 #pragma unroll
-        for (int b = 0; b < BPT; ++b) mst[b] = A.stat_exp ? scale_pow2_bf16<ELEM>(mb[b]) : mb[b];
-        const float G = row_pmean<BPT, TPR>(mst, A, C, redp, bar_id, wig, lane);
+          for (int b = 0; b < BPT; ++b) {
+            half_absmax_bits(xr[b], rot, mst[2 * b], mst[2 * b + 1]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t m = mst[2 * b + h];
+              if (A.stat_exp && m < 0x7F80u)
+                mst[2 * b + h] = __float_as_uint(e4m3_to_float(nvfp4_scale_code(bf16bits_to_float(m)))) >> 16;
+            }
+          }
+          G = row_pmean<2 * BPT, TPR>(mst, A, C, redp, bar_id, wig, lane);
+        } else {
+          uint32_t mst[BPT];
+#pragma unroll
+          for (int b = 0; b < BPT; ++b) mst[b] = A.stat_exp ? scale_pow2_bf16<ELEM>(mb[b]) : mb[b];
+          G = row_pmean<BPT, TPR>(mst, A, C, redp, bar_id, wig, lane);
+        }
         sc = (G == 0.0f) ? 0.0f : __frcp_rn(G);
         if (valid && tg == 0 && A.G_out) A.G_out[row] = G;
       }
@@ -576,14 +668,23 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
         }
         uint32_t qw[8];
         const uint64_t idx0 = (uint64_t)(row * (int64_t)C.D + (int64_t)k * kBlock);
-        const uint8_t code = quantise_block<SR, ELEM>(y, a, rot, idx0, pkeys, qw);
-        if (blk) {
-          if constexpr (ELEM == kElemE2M1)
+        if constexpr (ELEM == kElemNVFP4) {
+          (void)a;
+          const uint32_t codes2 = quantise_nvfp4<SR>(y, rot, idx0, pkeys, qw);
+          if (blk) {
             store_codes_e2m1(A.q + row * (int64_t)(C.D / 2) + (int64_t)k * (kBlock / 2), qw, rot);
-          else
-            store_codes(A.q + row * (int64_t)C.D + (int64_t)k * kBlock, qw, rot);
-          const int64_t so = A.scale_mma ? mma_scale_offset(row, k, A.kp4) : row * (int64_t)C.K + k;
-          A.scales[so] = code;
+            *reinterpret_cast<uint16_t*>(A.scales + row * (int64_t)(2 * C.K) + 2 * k) = (uint16_t)codes2;
+          }
+        } else {
+          const uint8_t code = quantise_block<SR, ELEM>(y, a, rot, idx0, pkeys, qw);
+          if (blk) {
+            if constexpr (ELEM == kElemE2M1)
+              store_codes_e2m1(A.q + row * (int64_t)(C.D / 2) + (int64_t)k * (kBlock / 2), qw, rot);
+            else
+              store_codes(A.q + row * (int64_t)C.D + (int64_t)k * kBlock, qw, rot);
+            const int64_t so = A.scale_mma ? mma_scale_offset(row, k, A.kp4) : row * (int64_t)C.K + k;
+            A.scales[so] = code;
+          }
         }
       }
     }

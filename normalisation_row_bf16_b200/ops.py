@@ -17,7 +17,7 @@ from . import build as _build
 
 RNE, SR = 0, 1
 SCALES_ROWMAJOR, SCALES_MMA = 0, 1
-ELEM = {"e4m3": 0, "e2m1": 1}
+ELEM = {"e4m3": 0, "e2m1": 1, "nvfp4": 2}
 STAT = {"absmax": 0, "scale_exp": 1}
 MXN_OK, MXN_ERR_ARG, MXN_ERR_UNSUPPORTED, MXN_ERR_CUDA, MXN_ERR_TIMEOUT = 0, -1, -2, -3, -4
 
@@ -110,7 +110,9 @@ def scales_bytes(T: int, D: int, layout: int = SCALES_ROWMAJOR) -> int:
 
 def _alloc_outputs(x, T, D, layout, q, scales, elem: str = "e4m3"):
     if q is None:
-        q = torch.empty(T, D // 2 if elem == "e2m1" else D, dtype=torch.uint8, device=x.device)
+        q = torch.empty(T, D if elem == "e4m3" else D // 2, dtype=torch.uint8, device=x.device)
+    if scales is None and elem == "nvfp4":
+        scales = torch.empty(T, D // 16, dtype=torch.uint8, device=x.device)
     if scales is None:
         n = scales_bytes(T, D, layout)
         scales = (torch.empty(T, D // 32, dtype=torch.uint8, device=x.device) if layout == SCALES_ROWMAJOR

@@ -150,7 +150,8 @@ def test_codes_bytes(L):
     assert L.mxnorm_codes_bytes(8192, 4096, 1) == 8192 * 2048
     assert L.mxnorm_codes_bytes(3, 96, 1) == 3 * 48
     assert L.mxnorm_codes_bytes(4, 33, 0) == 0
-    assert L.mxnorm_codes_bytes(4, 64, 2) == 0
+    assert L.mxnorm_codes_bytes(4, 64, 2) == 4 * 32        # NVFP4
+    assert L.mxnorm_codes_bytes(4, 64, 3) == 0
     assert L.mxnorm_codes_bytes(-1, 64, 0) == 0
 
 
@@ -158,7 +159,9 @@ def test_variant_entry_points_validate(L):
     st = None
     fx = L.mxnorm_fwd_ex
     # element format and statistic out of range
-    assert fx(FAKE, None, FAKE, FAKE, None, 4, 64, 64, 2.0, 0, 0, 0, 2, 0, st) == ops.MXN_ERR_ARG
+    assert fx(FAKE, None, FAKE, FAKE, None, 4, 64, 64, 2.0, 0, 0, 0, 3, 0, st) == ops.MXN_ERR_ARG
+    # NVFP4 scales exist only row-major
+    assert fx(FAKE, None, FAKE, FAKE, None, 4, 64, 64, 2.0, 0, 0, 1, 2, 0, st) == ops.MXN_ERR_UNSUPPORTED
     assert fx(FAKE, None, FAKE, FAKE, None, 4, 64, 64, 2.0, 0, 0, 0, 0, 3, st) == ops.MXN_ERR_ARG
     # the shared checks still apply
     assert fx(FAKE, None, FAKE, FAKE, None, 4, 33, 64, 2.0, 0, 0, 0, 1, 0, st) == ops.MXN_ERR_ARG

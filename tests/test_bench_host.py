@@ -20,6 +20,8 @@ def test_algorithmic_bytes_definitions():
     assert bench.algorithmic_bytes(T, D) == T * D * 2 + T * D + T * D // 32 + 2 * D + 4 * T == 101752832
     # MXFP4: half a byte per code
     assert bench.fp4_bytes(T, D) == T * D * 2 + T * D // 2 + T * D // 32 + 2 * D + 4 * T
+    # NVFP4: half a byte per code, one E4M3 scale per 16
+    assert bench.nvfp4_bytes(T, D) == T * D * 2 + T * D // 2 + T * D // 16 + 2 * D + 4 * T
     # two-pass comparator: RMSNorm reads x and writes y (bf16), the cast reads y
     # and writes codes and scales
     assert bench.two_pass_bytes(T, D) >= T * D * (2 + 2 + 2 + 1) + T * D // 32

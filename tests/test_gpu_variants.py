@@ -239,3 +239,67 @@ def test_fold_weight_full_qkv_sampled_rows():
     rows = np.random.default_rng(4).choice(6144, 64, replace=False)
     q_ref, s_ref = oracle.mx_cast(w.cpu(), g.cpu(), rows=rows)
     assert np.array_equal(to_np_u8(q)[rows], q_ref) and np.array_equal(to_np_u8(s)[rows], s_ref)
+
+
+# ------------------------------------------------------------------- NVFP4
+
+@pytest.mark.parametrize("T,D,kind", [(64, 1024, "normal"), (37, 4096, "outliers"), (5, 96, "student_t"),
+                                      (130, 2048, "student_t"), (9, 8192, "outliers"), (3, 16384, "normal")])
+@pytest.mark.parametrize("rounding", [ops.RNE, ops.SR])
+def test_nvfp4_forward(T, D, kind, rounding):
+    x = _dev(synthetic.activations(T, D, kind, seed=T + 2 * D))
+    g = _dev(synthetic.gamma(D, seed=T + 1))
+    q, s, G = ops.mxnorm_fwd_ex(x, g, 2.0, rounding=rounding, seed=31, elem="nvfp4")
+    torch.cuda.synchronize()
+    assert q.shape == (T, D // 2) and s.shape == (T, D // 16)
+    check_mxnorm_fwd(x, g, 2.0, rounding, 31, q, s, G, fmt="nvfp4")
+
+
+@pytest.mark.parametrize("p", [1.0, 4.0, math.inf, 2.5])
+@pytest.mark.parametrize("stat", ["absmax", "scale_exp"])
+def test_nvfp4_forward_p_stat_no_gamma(p, stat):
+    T, D = 50, 2080
+    x = _dev(synthetic.activations(T, D, "outliers", seed=5))
+    q, s, G = ops.mxnorm_fwd_ex(x, None, p, elem="nvfp4", stat=stat)
+    torch.cuda.synchronize()
+    check_mxnorm_fwd(x, None, p, ops.RNE, 0, q, s, G, fmt="nvfp4", stat=stat)
+
+
+@pytest.mark.parametrize("rounding", [ops.RNE, ops.SR])
+@pytest.mark.parametrize("with_gain", [False, True])
+def test_nvfp4_cast(rounding, with_gain):
+    T, D = 33, 4096
+    x = _dev(synthetic.activations(T, D, "student_t", seed=14))
+    gain = _dev(synthetic.gamma(D, seed=14)) if with_gain else None
+    q, s = ops.mx_cast(x, gain, rounding=rounding, seed=6, elem="nvfp4")
+    torch.cuda.synchronize()
+    check_cast(x, rounding, 6, q, s, gain_dev=gain, fmt="nvfp4")
+
+
+def test_nvfp4_zero_and_nonfinite_blocks():
+    T, D = 4, 128
+    x = synthetic.activations(T, D, "normal", seed=8)
+    x[1, 16:32] = 0.0
+    x[1, 48:64] = -0.0
+    x[2, 70] = float("nan")
+    x[3, 100] = float("-inf")
+    xd = _dev(x)
+    q, s = ops.mx_cast(xd, elem="nvfp4")
+    torch.cuda.synchronize()
+    check_cast(xd, ops.RNE, 0, q, s, fmt="nvfp4")
+    sh = to_np_u8(s)
+    assert sh[1, 1] == 0 and sh[1, 3] == 0 and sh[2, 4] == 0x7F and sh[3, 6] == 0x7F
+    with pytest.raises(ops.MXNormError):
+        ops.mxnorm_fwd_ex(xd, None, 2.0, elem="nvfp4", scale_layout=ops.SCALES_MMA)
+
+
+def test_nvfp4_llama8b_shape_sampled_rows():
+    w = synthetic.WORKLOADS["llama8b_8192x4096_outliers_p2"]
+    x = synthetic.activations(w["T"], w["D"], w["kind"], seed=0, device="cuda")
+    g = synthetic.gamma(w["D"], seed=0, device="cuda")
+    rows = np.concatenate([np.arange(0, 8), np.random.default_rng(3).choice(w["T"], 40, replace=False),
+                           np.arange(w["T"] - 8, w["T"])])
+    for rnd in (ops.RNE, ops.SR):
+        q, s, G = ops.mxnorm_fwd_ex(x, g, 2.0, rounding=rnd, seed=2, elem="nvfp4")
+        torch.cuda.synchronize()
+        check_mxnorm_fwd(x, g, 2.0, rnd, 2, q, s, G, rows=rows, strict=False, fmt="nvfp4")
