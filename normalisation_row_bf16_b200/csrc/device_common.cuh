@@ -6,7 +6,6 @@
 #pragma once
 
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -298,29 +297,36 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4_rn(float a, float b, float c, flo
 
 // ------------------------------------------------------------------ NVFP4 scale
 
-// fp32 value of a non-negative E4M3 code (0..0x7E), by the hardware decoder.
-__device__ __forceinline__ float e4m3_to_float(uint32_t c) {
-  uint32_t h2;
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
-      : "=r"(h2)
-      : "r"(c));
-  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+// The NVFP4 block scale: the smallest E4M3 value s with a <= 6 s (a >= 0
+// finite), 448 when even that is too small, returned as its exact fp32 value.
+// u = fl(a * c) with c the fp32 value just below 1/6 (6c = 1 - 2^-24, and a
+// rounding adds at most 2^-24 relative: (1 - 2^-24)(1 + 2^-24) < 1) is below
+// a / 6, so s is u rounded up onto the E4M3 grid -- 3 mantissa bits from 2^-6
+// up (an integer add and mask on the bits), multiples of 2^-9 below -- or the
+// next grid value when 6 s < a, which one exact comparison settles (6 s is
+// exact in fp32).  For a > 6 * 448 the result is clamped to 448.
+__device__ __forceinline__ float nvfp4_scale_value(float a) {
+  const float u = a * 0.16666665673255920f;
+  const uint32_t nb = (__float_as_uint(u) + 0xFFFFFu) & 0xFFF00000u;
+  const float sub = ceilf(u * 512.0f) * (1.0f / 512.0f);
+  const bool normal = u >= 0.015625f;
+  float s = normal ? __uint_as_float(nb) : sub;
+  const float next = normal ? __uint_as_float(nb + 0x100000u) : s + (1.0f / 512.0f);
+  s = (6.0f * s < a) ? next : s;
+  return fminf(s, 448.0f);
 }
 
-// The NVFP4 block scale: the E4M3 code of the smallest E4M3 value s with
-// a <= 6 s (a >= 0 finite), 0x7E when even 448 is too small.  The estimate
-// E4M3(a / 6) is within one code of it (E4M3's relative spacing is >= 1/16,
-// the estimate's error ~1e-7), and 6 s is exact in fp32, so one comparison
-// each way settles it.
-__device__ __forceinline__ uint32_t nvfp4_scale_code(float a) {
-  if (a > 2688.0f) return 0x7Eu;
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(a * (1.0f / 6.0f)));
-  uint32_t c = r & 0xFFu;
-  if (6.0f * e4m3_to_float(c) < a) c += 1;
-  else if (c > 0 && 6.0f * e4m3_to_float(c - 1) >= a) c -= 1;
-  return c > 0x7Eu ? 0x7Eu : c;
+// E4M3 code of an E4M3 value v >= 0 held exactly in fp32: (E - 127 + 7) << 3 |
+// mantissa from 2^-6 up; below, v = k * 2^-9 with k = 0..7, read off the bits
+// of v * 512 + 2^23.
+__device__ __forceinline__ uint32_t e4m3_code_of(float v) {
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t sub = __float_as_uint(fmaf(v, 512.0f, 8388608.0f)) - 0x4B000000u;
+  return b >= 0x3C800000u ? ((((b >> 23) - 120u) << 3) | ((b >> 20) & 7u)) : sub;
 }
+
+// The NVFP4 block scale as its E4M3 code.
+__device__ __forceinline__ uint32_t nvfp4_scale_code(float a) { return e4m3_code_of(nvfp4_scale_value(a)); }
 
 // ------------------------------------------------------------------ E2M1 cast
 

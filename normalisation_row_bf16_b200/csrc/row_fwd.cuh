@@ -331,10 +331,8 @@ __device__ __forceinline__ void half_absmax_bits(const uint32_t (&w)[16], int ro
 // half's absmax, 0x7F for a half holding NaN or infinity), then the E2M1
 // codes of fl32(y * fl32(1/s)); a zero scale gives zero codes, a NaN half
 // codes 0x7.  Returns the two scale codes (half 0 in bits 0..7).
-template <bool SR>
-__device__ __forceinline__ uint32_t quantise_nvfp4(const float (&y)[32], int rot, uint64_t idx0,
-                                                   const PhiloxKeys& pk, uint32_t (&qw)[8]) {
-  float sm[4];
+// Absmax of each 8-element slot of a block's y (slot order), NaN-propagating.
+__device__ __forceinline__ void slot_absmax(const float (&y)[32], float (&sm)[4]) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     float m0 = max3_abs_nan(0.0f, y[8 * j], y[8 * j + 1]);
@@ -343,14 +341,20 @@ __device__ __forceinline__ uint32_t quantise_nvfp4(const float (&y)[32], int rot
     m1 = max3_abs_nan(m1, y[8 * j + 6], y[8 * j + 7]);
     sm[j] = max3_abs_nan(m0, m1, 0.0f);
   }
+}
+
+template <bool SR>
+__device__ __forceinline__ uint32_t quantise_nvfp4(const float (&y)[32], const float (&sm)[4], int rot,
+                                                   uint64_t idx0, const PhiloxKeys& pk, uint32_t (&qw)[8]) {
   const float p01 = max3_abs_nan(sm[0], sm[1], 0.0f), p12 = max3_abs_nan(sm[1], sm[2], 0.0f);
   const float p23 = max3_abs_nan(sm[2], sm[3], 0.0f), p30 = max3_abs_nan(sm[3], sm[0], 0.0f);
   const float ah0 = rot == 0 ? p01 : (rot == 1 ? p30 : (rot == 2 ? p23 : p12));
   const float ah1 = rot == 0 ? p23 : (rot == 1 ? p12 : (rot == 2 ? p01 : p30));
   const bool bad0 = !(ah0 <= 3.402823466e38f), bad1 = !(ah1 <= 3.402823466e38f);   // NaN or infinity
-  const uint32_t c0 = bad0 ? 0x7Fu : nvfp4_scale_code(ah0), c1 = bad1 ? 0x7Fu : nvfp4_scale_code(ah1);
-  const float inv0 = (bad0 || c0 == 0) ? 0.0f : __frcp_rn(e4m3_to_float(c0));
-  const float inv1 = (bad1 || c1 == 0) ? 0.0f : __frcp_rn(e4m3_to_float(c1));
+  const float s0 = bad0 ? 0.0f : nvfp4_scale_value(ah0), s1 = bad1 ? 0.0f : nvfp4_scale_value(ah1);
+  const uint32_t c0 = bad0 ? 0x7Fu : e4m3_code_of(s0), c1 = bad1 ? 0x7Fu : e4m3_code_of(s1);
+  const float inv0 = (s0 == 0.0f) ? 0.0f : __frcp_rn(s0);
+  const float inv1 = (s1 == 0.0f) ? 0.0f : __frcp_rn(s1);
 #pragma unroll
   for (int sl = 0; sl < 4; ++sl) {
     const bool h1 = (((sl + rot) & 3) >> 1) != 0;
@@ -618,7 +622,7 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
             for (int h = 0; h < 2; ++h) {
               const uint32_t m = mst[2 * b + h];
               if (A.stat_exp && m < 0x7F80u)
-                mst[2 * b + h] = __float_as_uint(e4m3_to_float(nvfp4_scale_code(bf16bits_to_float(m)))) >> 16;
+                mst[2 * b + h] = __float_as_uint(nvfp4_scale_value(bf16bits_to_float(m))) >> 16;
             }
           }
           G = row_pmean<2 * BPT, TPR>(mst, A, C, redp, bar_id, wig, lane);
@@ -639,20 +643,28 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
         const int kk = k < C.K ? k : C.K - 1;          // in-range gamma reads
         float y[32];
         float a;
+        float sm[4];                                   // NVFP4: per-slot maxima of y
         if constexpr (has_gamma) {
           float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             float2 gf[4];
             gamma_slot<kGF32>(smem, C.K, j, kk, gf);
+            float b0 = 0.0f, b1 = 0.0f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float2 yv = mul2(mul2(bf16x2_to_f2(xr[b][4 * j + i]), s2), gf[i]);
               y[8 * j + 2 * i] = yv.x;
               y[8 * j + 2 * i + 1] = yv.y;
-              if (i & 1) a1 = max3_abs_nan(a1, yv.x, yv.y);
-              else a0 = max3_abs_nan(a0, yv.x, yv.y);
+              if constexpr (ELEM == kElemNVFP4) {
+                if (i & 1) b1 = max3_abs_nan(b1, yv.x, yv.y);
+                else b0 = max3_abs_nan(b0, yv.x, yv.y);
+              } else {
+                if (i & 1) a1 = max3_abs_nan(a1, yv.x, yv.y);
+                else a0 = max3_abs_nan(a0, yv.x, yv.y);
+              }
             }
+            if constexpr (ELEM == kElemNVFP4) sm[j] = max3_abs_nan(b0, b1, 0.0f);
           }
           a = max3_abs_nan(a0, a1, 0.0f);
         } else {
@@ -670,7 +682,8 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
         const uint64_t idx0 = (uint64_t)(row * (int64_t)C.D + (int64_t)k * kBlock);
         if constexpr (ELEM == kElemNVFP4) {
           (void)a;
-          const uint32_t codes2 = quantise_nvfp4<SR>(y, rot, idx0, pkeys, qw);
+          if constexpr (!has_gamma) slot_absmax(y, sm);
+          const uint32_t codes2 = quantise_nvfp4<SR>(y, sm, rot, idx0, pkeys, qw);
           if (blk) {
             store_codes_e2m1(A.q + row * (int64_t)(C.D / 2) + (int64_t)k * (kBlock / 2), qw, rot);
             *reinterpret_cast<uint16_t*>(A.scales + row * (int64_t)(2 * C.K) + 2 * k) = (uint16_t)codes2;
