@@ -383,17 +383,6 @@ __device__ __forceinline__ void philox4x32_10_x2(uint4& a, uint4& b, const Philo
   }
 }
 
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys& K) {
-  constexpr uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
-#pragma unroll
-  for (int r = 0; r < 10; ++r) {
-    const uint64_t p0 = (uint64_t)M0 * c.x, p1 = (uint64_t)M1 * c.z;
-    c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ K.k0[r], (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ K.k1[r],
-                   (uint32_t)p0);
-  }
-  return c;
-}
-
 // Stochastic rounding of v (|v| <= 448, finite) onto the E4M3 grid, returned
 // as the fp32 grid value (exact) with v's sign.  lo = the grid value at or
 // below |v|, step = grid spacing there; up iff r < (|v| - lo) / step * 2^32.

@@ -254,14 +254,15 @@ __device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a,
       if constexpr (SR) {
         const int c = (sl + rot) & 3;
         const uint64_t ctr = (idx0 + (uint64_t)(c * 8)) >> 2;
+        uint4 rr[2] = {make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), 0u, 0u),
+                       make_uint4((uint32_t)(ctr + 1), (uint32_t)((ctr + 1) >> 32), 0u, 0u)};
+        philox4x32_10_x2(rr[0], rr[1], pk);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const uint64_t cc = ctr + h;
-          const uint4 r = philox4x32_10(make_uint4((uint32_t)cc, (uint32_t)(cc >> 32), 0u, 0u), pk);
-          v[4 * h] = sr_e2m1_grid(v[4 * h], r.x);
-          v[4 * h + 1] = sr_e2m1_grid(v[4 * h + 1], r.y);
-          v[4 * h + 2] = sr_e2m1_grid(v[4 * h + 2], r.z);
-          v[4 * h + 3] = sr_e2m1_grid(v[4 * h + 3], r.w);
+          v[4 * h] = sr_e2m1_grid(v[4 * h], rr[h].x);
+          v[4 * h + 1] = sr_e2m1_grid(v[4 * h + 1], rr[h].y);
+          v[4 * h + 2] = sr_e2m1_grid(v[4 * h + 2], rr[h].z);
+          v[4 * h + 3] = sr_e2m1_grid(v[4 * h + 3], rr[h].w);
         }
       }
       qw[sl] = nan_block ? 0x77777777u : cvt_e2m1x8_rn(v);
