@@ -245,7 +245,8 @@ size_t mxnorm_bwd_workspace_size(int64_t T, int64_t D);
  * b_s   uint8 scales of B in the MXN_SCALES_MMA layout (N x K/32 bytes)
  * c     bf16 [M, N] row-major (written)
  * Requires M % 128 == 0, N % 256 == 0, K % 128 == 0 (MXN_ERR_UNSUPPORTED
- * otherwise); M = 0 or N = 0 is a no-op.  One CTA per 128 x 256 tile.
+ * otherwise); M = 0 or N = 0 is a no-op.  Persistent CTAs, one per SM,
+ * walk the 128 x 256 output tiles.
  */
 int mxfp8_gemm(const void* a_q, const void* a_s, const void* b_q, const void* b_s, void* c, int64_t M,
                int64_t N, int64_t K, void* stream);
@@ -288,9 +289,10 @@ int mxnorm_device_status(void* stream);
 
 /*
  * Launch tuning for the row kernels: threads per CTA (a multiple of 32 up to
- * 512; the forward kernels split them into row groups, the backward uses them
- * as consumer threads and accepts 128, 256 or 512), shared-memory stages per
- * pipeline (1..16) and CTAs per SM (1..8); 0 keeps the library's choice.
+ * 512, split into row groups; capped at what the kernel's register budget
+ * allows -- 512 for most shapes, 256 for the backward's two-block rows),
+ * shared-memory stages per row group (1..16) and CTAs per SM (1..8); 0 keeps
+ * the library's choice.
  * Process-wide; not thread-safe against concurrent launches.  Returns
  * MXN_ERR_ARG for out-of-range values; a shape that does not fit an SM makes
  * the next launch return MXN_ERR_UNSUPPORTED.

@@ -425,7 +425,7 @@ int launch_bwd(const BwdPlan& P, const BwdArgs& A, uint16_t* dgamma, cudaStream_
 
 // ----------------------------------------------- allocation-free backward
 //
-// Scratch for mxnorm_bwd_noalloc: the per-CTA dgamma partial sums, 2^21 fp32
+// Scratch for mxnorm_bwd_noalloc: the per-row-group dgamma partial sums, 2^21 fp32
 // (8 MiB).  Every device that loads this library holds it until the process
 // exits.  In host code the name is only a host-side stand-in; its device
 // address comes from cudaGetSymbolAddress, looked up once per device with
