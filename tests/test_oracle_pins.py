@@ -19,6 +19,9 @@
   orthogonality x . dx = 0, linearity in gamma.
 * RMSNorm: torch.nn.functional.rms_norm in float64 rounded to bf16.
 * GEMM entries: torch dequantisation (float8 decoders) and float64 matmul.
+* Brute force on tiny rows: every assignment of a small value set to three
+  columns of a two-block row, against the closed-form G and a Python
+  evaluation of the definitions (scale by scanning e, nearest-grid codes).
 """
 import math
 import os
@@ -467,3 +470,54 @@ def test_gemm_entries_vs_torch_dequant():
     ii, jj = np.meshgrid(np.arange(M), np.arange(N), indexing="ij")
     c = oracle.mxfp8_gemm_entries(aq, a_s, bq, b_s, ii.ravel(), jj.ravel())
     assert np.allclose(c.reshape(M, N), ref.numpy(), rtol=1e-12, atol=1e-300)
+
+
+def _brute_row(xrow, G, gamma=None):
+    """Codes and scales of one row from the definitions, in Python: y by numpy
+    float32 operations, the scale by scanning e, codes by nearest-grid search
+    (ties to the even code) on the E4M3 grid."""
+    s = np.float32(0.0) if G == 0 else np.float32(1.0) / np.float32(G)
+    y = (xrow.astype(np.float32) * s).astype(np.float32)
+    if gamma is not None:
+        y = (y * gamma.astype(np.float32)).astype(np.float32)
+    codes, scales = [], []
+    for k in range(y.size // 32):
+        blk = y[32 * k:32 * (k + 1)]
+        a = float(np.max(np.abs(blk.astype(np.float64))))
+        e = next(e for e in range(-127, 128) if a <= 448.0 * 2.0 ** e)
+        scales.append(e + 127)
+        v = (blk * np.float32(2.0 ** -e)).astype(np.float32).astype(np.float64)
+        av = np.minimum(np.abs(v), 448.0)
+        d = np.abs(av[:, None] - E4M3_GRID[None, :])
+        best = d.min(axis=1, keepdims=True)
+        cand = d == best
+        even = cand & (np.arange(E4M3_GRID.size)[None, :] % 2 == 0)
+        idx = np.where(cand.sum(1) > 1, even.argmax(1), cand.argmax(1))
+        codes.append((idx | np.where(np.signbit(v), 0x80, 0)).astype(np.uint8))
+    return np.concatenate(codes), np.array(scales, np.uint8)
+
+
+def test_brute_force_tiny_rows_every_pattern():
+    """D = 64 (K = 2): every assignment of {0, 1, -1.5, 3.25, -96, 2^-20} to
+    columns 0, 5 (block 0) and 40 (block 1), the rest zero; p = 2 and inf,
+    without and with a gain.  G against the closed form, codes and scales
+    against the brute-force row."""
+    import itertools
+    vals = [0.0, 1.0, -1.5, 3.25, -96.0, 2.0 ** -20]
+    rows = []
+    for a, b, c in itertools.product(vals, repeat=3):
+        r = np.zeros(64, np.float32)
+        r[0], r[5], r[40] = a, b, c
+        rows.append(r)
+    x = torch.from_numpy(np.stack(rows)).to(torch.bfloat16)
+    xf = x.float().numpy()
+    gam = torch.from_numpy((1.0 + 0.25 * np.arange(64) / 64).astype(np.float32)).to(torch.bfloat16)
+    for p in (2.0, math.inf):
+        for g in (None, gam):
+            q, s, G = oracle.mxnorm_fwd(x, g, p)
+            for t in range(xf.shape[0]):
+                m = np.abs(xf[t].astype(np.float64)).reshape(2, 32).max(1)
+                Gw = m.max() if math.isinf(p) else math.sqrt((m[0] ** 2 + m[1] ** 2) / 2)
+                assert abs(float(G[t]) - Gw) <= 6e-8 * Gw
+                qb, sb = _brute_row(xf[t], G[t], None if g is None else g.float().numpy())
+                assert np.array_equal(q[t], qb) and np.array_equal(s[t], sb), (p, t)
