@@ -546,6 +546,7 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
 
     // ---- pass 1: block maxima (MXNorm, Cast) or sum of squares (RMSNorm)
     uint32_t mb[BPT];
+    uint32_t mh[BPT][2];                      // NVFP4: the two 16-element halves
     float2 ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int b = 0; b < BPT; ++b) {
@@ -564,6 +565,9 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
             }
           }
         }
+      } else if constexpr (ELEM == kElemNVFP4) {
+        half_absmax_bits(xr[b], rot, mh[b][0], mh[b][1]);   // NVFP4 blocks are the halves
+        mb[b] = max(mh[b][0], mh[b][1]);
       } else {
         mb[b] = block_absmax16(xr[b]);
       }
@@ -618,7 +622,8 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
           uint32_t mst[2 * BPT];
 #pragma unroll
           for (int b = 0; b < BPT; ++b) {
-            half_absmax_bits(xr[b], rot, mst[2 * b], mst[2 * b + 1]);
+            mst[2 * b] = mh[b][0];
+            mst[2 * b + 1] = mh[b][1];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const uint32_t m = mst[2 * b + h];
