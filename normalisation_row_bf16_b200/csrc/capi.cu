@@ -415,9 +415,20 @@ int launch_bwd(const BwdPlan& P, const BwdArgs& A, uint16_t* dgamma, cudaStream_
   int rc = launch_pdl(P.kernel, P.grid, P.threads, P.smem, argv, s, "row_bwd_kernel launch");
   if (rc) return rc;
   if (A.partial) {
-    dgamma_reduce_kernel<<<(unsigned)((P.C.D + 31) / 32), dim3(32, 32), 0, s>>>(
-        A.partial, (int64_t)P.partial_rows(), P.C.D, dgamma);
-    const cudaError_t e = cudaGetLastError();
+    const float* part = A.partial;
+    int64_t n_part = (int64_t)P.partial_rows();
+    int D = P.C.D;
+    void* rargv[] = {&part, &n_part, &D, &dgamma};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((D + 31) / 32));
+    cfg.blockDim = dim3(32, 32);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelExC(&cfg, (const void*)dgamma_reduce_kernel, rargv);
     if (e != cudaSuccess) return cuda_fail(e, "dgamma_reduce_kernel launch");
   }
   return MXN_OK;

@@ -184,6 +184,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
+  // Programmatic dependent launch: the set-up above overlaps the previous
+  // kernel's tail; operands are read and C written only after it completed.
+  griddep_wait();
+  griddep_launch_dependents();
 
   uint32_t n_issued = 0;                        // producer: stages issued
   if (warp == 0) {
@@ -369,11 +373,21 @@ int gemm_mxfp8_launch(const void* a_q, const void* a_s, const void* b_q, const v
   cudaError_t e = cudaFuncSetAttribute(gemm_mxfp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) { *why = cudaGetErrorString(e); return (int)e; }
   const int tiles = (M / kTileM) * (N / kTileN);
-  dim3 grid(tiles < sms ? tiles : sms);
-  gemm_mxfp8_kernel<<<grid, kThreads, smem, stream>>>(ma, mb, static_cast<const uint8_t*>(a_s),
-                                                      static_cast<const uint8_t*>(b_s),
-                                                      static_cast<uint16_t*>(c), M, N, K, status);
-  e = cudaGetLastError();
+  const uint8_t* as = static_cast<const uint8_t*>(a_s);
+  const uint8_t* bs = static_cast<const uint8_t*>(b_s);
+  uint16_t* cp = static_cast<uint16_t*>(c);
+  void* argv[] = {&ma, &mb, &as, &bs, &cp, &M, &N, &K, &status};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tiles < sms ? tiles : sms);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelExC(&cfg, (const void*)gemm_mxfp8_kernel, argv);
   if (e != cudaSuccess) { *why = cudaGetErrorString(e); return (int)e; }
   return 0;
 }

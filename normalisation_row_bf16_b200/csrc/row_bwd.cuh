@@ -304,6 +304,7 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
 __global__ void __launch_bounds__(1024) dgamma_reduce_kernel(const float* partial, int64_t n_part,
                                                              int D, uint16_t* dgamma) {
   __shared__ float sh[32][33];
+  griddep_wait();                  // the backward kernel's partial rows are complete
   const int tx = threadIdx.x, ty = threadIdx.y;
   const int j = blockIdx.x * 32 + tx;
   float s = 0.0f;
