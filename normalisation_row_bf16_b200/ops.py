@@ -108,15 +108,31 @@ def scales_bytes(T: int, D: int, layout: int = SCALES_ROWMAJOR) -> int:
     return int(lib().mxnorm_scales_bytes(T, D, layout))
 
 
+def _check_buffer(t, name, nbytes, dtype, device):
+    """A caller-provided output must hold the bytes the library will write
+    (the C ABI takes raw pointers and cannot check)."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor")
+    if t.numel() * t.element_size() < nbytes:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, {nbytes} needed")
+
+
 def _alloc_outputs(x, T, D, layout, q, scales, elem: str = "e4m3"):
+    q_bytes = T * (D if elem == "e4m3" else D // 2)
+    s_bytes = T * (D // 16) if elem == "nvfp4" else scales_bytes(T, D, layout)
+    _check_buffer(q, "q", q_bytes, torch.uint8, x.device)
+    _check_buffer(scales, "scales", s_bytes, torch.uint8, x.device)
     if q is None:
         q = torch.empty(T, D if elem == "e4m3" else D // 2, dtype=torch.uint8, device=x.device)
     if scales is None and elem == "nvfp4":
         scales = torch.empty(T, D // 16, dtype=torch.uint8, device=x.device)
     if scales is None:
-        n = scales_bytes(T, D, layout)
         scales = (torch.empty(T, D // 32, dtype=torch.uint8, device=x.device) if layout == SCALES_ROWMAJOR
-                  else torch.zeros(max(n, 1), dtype=torch.uint8, device=x.device))
+                  else torch.zeros(max(s_bytes, 1), dtype=torch.uint8, device=x.device))
     return q, scales
 
 
@@ -126,6 +142,7 @@ def mxnorm_fwd(x, gamma=None, p: float = 2.0, rounding: int = RNE, seed: int = 0
     T, D, ld = _rows_ld(x)
     gamma = _bf16_vec(gamma, D)
     q, scales = _alloc_outputs(x, T, D, scale_layout, q, scales)
+    _check_buffer(G, "G", 4 * T, torch.float32, x.device)
     if G is None:
         G = torch.empty(T, dtype=torch.float32, device=x.device)
     _check(lib().mxnorm_fwd(_ptr(x), _ptr(gamma), _ptr(q), _ptr(scales), _ptr(G), T, D, ld,
@@ -152,6 +169,7 @@ def mxnorm_fwd_ex(x, gamma=None, p: float = 2.0, rounding: int = RNE, seed: int 
     T, D, ld = _rows_ld(x)
     gamma = _bf16_vec(gamma, D)
     q, scales = _alloc_outputs(x, T, D, scale_layout, q, scales, elem)
+    _check_buffer(G, "G", 4 * T, torch.float32, x.device)
     if G is None:
         G = torch.empty(T, dtype=torch.float32, device=x.device)
     _check(lib().mxnorm_fwd_ex(_ptr(x), _ptr(gamma), _ptr(q), _ptr(scales), _ptr(G), T, D, ld,
@@ -187,6 +205,7 @@ def fold_weight(w, gamma, elem: str = "e4m3", scale_layout: int = SCALES_MMA, q=
 def rmsnorm_bf16(x, gamma=None, eps: float = 1e-5, y=None, stream=None):
     T, D, ld = _rows_ld(x)
     gamma = _bf16_vec(gamma, D)
+    _check_buffer(y, "y", 2 * T * D, torch.bfloat16, x.device)
     if y is None:
         y = torch.empty(T, D, dtype=torch.bfloat16, device=x.device)
     _check(lib().rmsnorm_bf16(_ptr(x), _ptr(gamma), _ptr(y), T, D, ld, float(eps), _stream(stream)))
@@ -199,6 +218,7 @@ def rmsnorm_then_mxcast(x, gamma=None, eps: float = 1e-5, scale_layout: int = SC
     T, D, ld = _rows_ld(x)
     gamma = _bf16_vec(gamma, D)
     q, scales = _alloc_outputs(x, T, D, scale_layout, q, scales)
+    _check_buffer(y_tmp, "y_tmp", 2 * T * D, torch.bfloat16, x.device)
     if y_tmp is None:
         y_tmp = torch.empty(T, D, dtype=torch.bfloat16, device=x.device)
     _check(lib().rmsnorm_then_mxcast(_ptr(x), _ptr(gamma), float(eps), _ptr(y_tmp), _ptr(q),
@@ -217,6 +237,9 @@ def mxnorm_bwd(x, dy, gamma, G, dx=None, dgamma=None, workspace=None, want_dgamm
     if ld != D or dy.shape != x.shape or not dy.is_contiguous() or dy.dtype != torch.bfloat16:
         raise ValueError("x and dy must be dense bf16 [T, D]")
     gamma = _bf16_vec(gamma, D)
+    _check_buffer(G, "G", 4 * T, torch.float32, x.device)
+    _check_buffer(dx, "dx", 2 * T * D, torch.bfloat16, x.device)
+    _check_buffer(dgamma, "dgamma", 2 * D, torch.bfloat16, x.device)
     if dx is None:
         dx = torch.empty_like(x)
     if gamma is not None and want_dgamma and dgamma is None:
@@ -226,6 +249,7 @@ def mxnorm_bwd(x, dy, gamma, G, dx=None, dgamma=None, workspace=None, want_dgamm
         nbytes = bwd_workspace_bytes(T, D)
         if workspace is None:
             workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+        _check_buffer(workspace, "workspace", 0, workspace.dtype, x.device)
         nbytes = workspace.numel() * workspace.element_size()
     _check(lib().mxnorm_bwd(_ptr(x), _ptr(dy), _ptr(gamma), _ptr(G), _ptr(dx), _ptr(dgamma), T, D,
                             _ptr(workspace), nbytes, _stream(stream)))
@@ -241,6 +265,9 @@ def mxnorm_bwd_noalloc(x, dy, gamma, G, dx=None, dgamma=None, want_dgamma: bool 
     if ld != D or dy.shape != x.shape or not dy.is_contiguous() or dy.dtype != torch.bfloat16:
         raise ValueError("x and dy must be dense bf16 [T, D]")
     gamma = _bf16_vec(gamma, D)
+    _check_buffer(G, "G", 4 * T, torch.float32, x.device)
+    _check_buffer(dx, "dx", 2 * T * D, torch.bfloat16, x.device)
+    _check_buffer(dgamma, "dgamma", 2 * D, torch.bfloat16, x.device)
     if dx is None:
         dx = torch.empty_like(x)
     if gamma is not None and want_dgamma and dgamma is None:
@@ -257,6 +284,9 @@ def mxfp8_gemm(a_q, a_s, b_q, b_s, M: int, N: int, K: int, c=None, stream=None):
             raise ValueError("GEMM operands must be uint8 CUDA tensors")
     if a_q.numel() != M * K or b_q.numel() != N * K:
         raise ValueError("code tensors do not match M, N, K")
+    _check_buffer(a_s, "a_s", scales_bytes(M, K, SCALES_MMA), torch.uint8, a_q.device)
+    _check_buffer(b_s, "b_s", scales_bytes(N, K, SCALES_MMA), torch.uint8, a_q.device)
+    _check_buffer(c, "c", 2 * M * N, torch.bfloat16, a_q.device)
     if c is None:
         c = torch.empty(M, N, dtype=torch.bfloat16, device=a_q.device)
     _check(lib().mxfp8_gemm(_ptr(a_q), _ptr(a_s), _ptr(b_q), _ptr(b_s), _ptr(c), M, N, K, _stream(stream)))

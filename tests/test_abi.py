@@ -187,3 +187,16 @@ def test_python_variant_bindings_refuse_cpu_tensors(L):
         ops.mx_cast(x)
     with pytest.raises(ValueError):
         ops.fold_weight(x, x[0])
+
+
+def test_binding_checks_output_buffers(L):
+    """Caller-provided outputs must be CUDA tensors of the right type and size
+    on the input's device (the C ABI writes through raw pointers)."""
+    import torch
+    from normalisation_row_bf16_b200.ops import _check_buffer
+    cuda0 = torch.device("cuda", 0)
+    with pytest.raises(ValueError):
+        _check_buffer(torch.empty(10, dtype=torch.uint8), "q", 8, torch.uint8, cuda0)   # a CPU tensor
+    with pytest.raises(ValueError):
+        _check_buffer([0] * 10, "q", 8, torch.uint8, cuda0)                            # not a tensor
+    _check_buffer(None, "q", 8, torch.uint8, cuda0)                                     # allocated by the binding

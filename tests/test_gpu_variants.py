@@ -303,3 +303,25 @@ def test_nvfp4_llama8b_shape_sampled_rows():
         q, s, G = ops.mxnorm_fwd_ex(x, g, 2.0, rounding=rnd, seed=2, elem="nvfp4")
         torch.cuda.synchronize()
         check_mxnorm_fwd(x, g, 2.0, rnd, 2, q, s, G, rows=rows, strict=False, fmt="nvfp4")
+
+
+def test_binding_rejects_undersized_outputs():
+    x = _dev(synthetic.activations(4, 64, "normal", seed=0))
+    with pytest.raises(ValueError):
+        ops.mxnorm_fwd(x, q=torch.empty(4, 32, dtype=torch.uint8, device="cuda"))
+    with pytest.raises(ValueError):
+        ops.mxnorm_fwd(x, G=torch.empty(3, dtype=torch.float32, device="cuda"))
+    with pytest.raises(ValueError):
+        ops.mxnorm_fwd(x, q=torch.empty(4, 64, dtype=torch.int8, device="cuda"))
+    with pytest.raises(ValueError):
+        ops.mxnorm_fwd_ex(x, elem="nvfp4", scales=torch.empty(4, 2, dtype=torch.uint8, device="cuda"))
+    with pytest.raises(ValueError):
+        ops.mxnorm_fwd(x, scale_layout=ops.SCALES_MMA, scales=torch.empty(64, dtype=torch.uint8, device="cuda"))
+    dy = _dev(synthetic.upstream_grad(4, 64, seed=0))
+    _, _, G = ops.mxnorm_fwd(x)
+    with pytest.raises(ValueError):
+        ops.mxnorm_bwd(x, dy, None, G, dx=torch.empty(4, 32, dtype=torch.bfloat16, device="cuda"))
+    # right-sized buffers pass and are used in place
+    q = torch.empty(4, 64, dtype=torch.uint8, device="cuda")
+    q2, _, _ = ops.mxnorm_fwd(x, q=q)
+    assert q2.data_ptr() == q.data_ptr()
