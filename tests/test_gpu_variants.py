@@ -8,6 +8,8 @@
   folded chain MXNorm(gamma = NULL) -> GEMM(folded weight) against the oracle's
   chain entry by entry, and against the unfolded chain within quantisation
   error.
+* Every finite bf16 value through the FP4 casts, and every finite bf16
+  magnitude as a block's absmax under each format's scale rule.
 """
 import math
 
@@ -291,6 +293,66 @@ def test_nvfp4_zero_and_nonfinite_blocks():
     assert sh[1, 1] == 0 and sh[1, 3] == 0 and sh[2, 4] == 0x7F and sh[3, 6] == 0x7F
     with pytest.raises(ops.MXNormError):
         ops.mxnorm_fwd_ex(xd, None, 2.0, elem="nvfp4", scale_layout=ops.SCALES_MMA)
+
+
+def _finite_bf16_values(positive_only=False):
+    bits = np.arange(65536, dtype=np.uint32)
+    keep = ((bits >> 7) & 0xFF) != 0xFF
+    if positive_only:
+        keep &= bits < 0x8000
+    return torch.from_numpy(bits[keep].astype(np.uint16).view(np.int16)).view(torch.bfloat16).float()
+
+
+@pytest.mark.parametrize("elem", ["e2m1", "nvfp4"])
+def test_fp4_cast_every_bf16_pattern(elem):
+    """Every finite bf16 value through the FP4 casts: each block of 32 holds one
+    anchor that fixes the scale(s) and 31 test values, at several anchors, so
+    the E2M1 conversion of every bf16 magnitude is compared with the oracle's
+    rounding under MX (E8M0) and NVFP4 (E4M3) scales, nearest-even and
+    stochastic."""
+    vals = _finite_bf16_values()
+    rows = []
+    for anchor in (6.0, 2.0**100, 2.0**-100, 1.0, 3.0e38, 2688.0):
+        n = vals.numel()
+        nb = (n + 30) // 31
+        blk = torch.zeros(nb, 32)
+        blk[:, 0] = anchor
+        flat = torch.zeros(nb * 31)
+        flat[:n] = vals.clamp(-anchor, anchor)
+        blk[:, 1:] = flat.view(nb, 31)
+        rows.append(blk.reshape(-1))
+    x = torch.cat(rows)
+    x = x[: x.numel() // 1024 * 1024].view(-1, 1024).to(torch.bfloat16)
+    xd = _dev(x)
+    for rounding in (ops.RNE, ops.SR):
+        q, s = ops.mx_cast(xd, rounding=rounding, seed=9, elem=elem)
+        torch.cuda.synchronize()
+        check_cast(xd, rounding, 9, q, s, fmt=elem)
+
+
+@pytest.mark.parametrize("elem", ["e4m3", "e2m1", "nvfp4"])
+def test_block_scale_every_bf16_amax(elem):
+    """Every finite non-negative bf16 magnitude as the absmax of its own block
+    (at a random position, random sign, the other elements random fractions of
+    it), so each format's scale rule meets every bf16 amax, including the
+    E4M3-subnormal and saturated NVFP4 scales and the E8M0 boundaries."""
+    amax = _finite_bf16_values(positive_only=True)
+    B = 16 if elem == "nvfp4" else 32
+    nb = amax.numel()
+    rng = torch.Generator().manual_seed(11)
+    frac = torch.rand(nb, B, generator=rng) * 2.0 - 1.0
+    blk = (amax[:, None] * frac).to(torch.bfloat16).float()
+    pos = torch.randint(0, B, (nb,), generator=rng)
+    sign = torch.where(torch.rand(nb, generator=rng) < 0.5, -1.0, 1.0)
+    blk[torch.arange(nb), pos] = amax * sign
+    x = blk.reshape(-1)
+    pad = (-x.numel()) % 1024
+    x = torch.cat([x, torch.zeros(pad)]).view(-1, 1024).to(torch.bfloat16)
+    xd = _dev(x)
+    for rounding in (ops.RNE, ops.SR):
+        q, s = ops.mx_cast(xd, rounding=rounding, seed=12, elem=elem)
+        torch.cuda.synchronize()
+        check_cast(xd, rounding, 12, q, s, fmt=elem)
 
 
 def test_nvfp4_llama8b_shape_sampled_rows():
