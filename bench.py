@@ -407,6 +407,30 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
                                bwd_bytes(T, D, wsb.numel()), "row_bwd_kernel + dgamma_reduce_kernel")
     del dys, dxs, Gbs
 
+    # Size context for the headline's roofline fraction: the measured HBM peak
+    # is torch's copy_ over 4 GiB moved; the same copy_ moving only the
+    # forward's algorithmic bytes (half read, half written), and torch's
+    # elementwise bf16 -> float8_e4m3fn cast of x (reads 2 B, writes 1 B per
+    # element: the forward's byte pattern with no statistic and no block
+    # scales), show what a plain streaming kernel reaches at this size.  Sets
+    # rotate as above.
+    half = algorithmic_bytes(T, D) // 2 // 16 * 16
+    srcs = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(n_sets)]
+    dsts = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(n_sets)]
+    ctx = {"copy_same_bytes": run_graph_leg(args, world, dev, barrier,
+                                            lambda i: dsts[i % n_sets].copy_(srcs[i % n_sets]), 2 * half,
+                                            "torch copy_ (uint8), read + write bytes")}
+    del srcs, dsts
+    f8s = [torch.empty(T, D, dtype=torch.float8_e4m3fn, device=dev) for _ in range(n_sets)]
+    ctx["cast_bf16_to_e4m3"] = run_graph_leg(args, world, dev, barrier,
+                                             lambda i: f8s[i % n_sets].copy_(xs[i % n_sets]), 3 * T * D,
+                                             "torch elementwise cast bf16 -> float8_e4m3fn of x (no scales)")
+    del f8s
+    for v in ctx.values():
+        v["headline_over_this"] = round(v["ms"] / ms_per_step * algorithmic_bytes(T, D) / v["roofline"]
+                                        ["algorithmic_bytes_per_launch"], 3)
+    out["stream_context"] = ctx
+
     # Variants on the same batch: MXFP4 codes, the scale-reuse statistic.
     outs4 = [(torch.empty(T, D // 2, dtype=torch.uint8, device=dev),
               torch.empty(T, D // 32, dtype=torch.uint8, device=dev),
