@@ -216,6 +216,7 @@ def _c_limit(p, B=32):
 def test_theorem1_pmean_over_rms_converges_to_c():
     assert _c_limit(1.0) == pytest.approx(2.3470, abs=2e-3)
     assert _c_limit(2.0) == pytest.approx(2.3895, abs=2e-3)
+    assert _c_limit(4.0) == pytest.approx(2.4774, abs=2e-3)
     D = 1 << 20
     x = synthetic.activations(1, D, "normal", seed=11)
     rms = float(torch.sqrt((x.double() ** 2).mean()))
