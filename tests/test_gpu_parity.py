@@ -83,6 +83,20 @@ def test_mxnorm_fwd_sr_bit_exact(p):
         check_mxnorm_fwd(xd, gd, p, 1, seed, q, s, G, strict=False)
 
 
+@pytest.mark.parametrize("T,D", [(1, 32), (3, 96), (5, 160), (64, 64), (130, 544), (257, 1056), (33, 2080),
+                                 (7, 8192), (2, 32768)])
+def test_mxnorm_fwd_sr_ragged(T, D):
+    """Stochastic rounding at every launch shape it plans: rows sharing a warp
+    (up to 32 blocks), one block per thread (33..64), two (65..512) and four
+    (up to the 32768-column maximum)."""
+    x = synthetic.activations(T, D, "student_t", seed=T + D)
+    g = synthetic.gamma(D, seed=D)
+    xd, gd = _dev(x), _dev(g)
+    q, s, G = ops.mxnorm_fwd(xd, gd, 2.0, rounding=ops.SR, seed=D)
+    torch.cuda.synchronize()
+    check_mxnorm_fwd(xd, gd, 2.0, ops.SR, D, q, s, G, strict=False)
+
+
 def test_mxnorm_fwd_special_rows():
     D = 1024
     x = torch.zeros(8, D, dtype=torch.bfloat16)

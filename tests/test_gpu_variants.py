@@ -43,7 +43,8 @@ def _dev(t):
 # ------------------------------------------------------------------- MXFP4
 
 @pytest.mark.parametrize("T,D,kind", [(64, 1024, "normal"), (37, 4096, "outliers"), (5, 96, "student_t"),
-                                      (130, 2048, "student_t"), (9, 8192, "outliers"), (3, 16384, "normal")])
+                                      (130, 2048, "student_t"), (9, 8192, "outliers"), (3, 16384, "normal"),
+                                      (1, 32, "normal"), (33, 2080, "student_t"), (2, 32768, "student_t")])
 @pytest.mark.parametrize("rounding", [ops.RNE, ops.SR])
 def test_mxfp4_forward(T, D, kind, rounding):
     x = _dev(synthetic.activations(T, D, kind, seed=T + D))
@@ -246,7 +247,8 @@ def test_fold_weight_full_qkv_sampled_rows():
 # ------------------------------------------------------------------- NVFP4
 
 @pytest.mark.parametrize("T,D,kind", [(64, 1024, "normal"), (37, 4096, "outliers"), (5, 96, "student_t"),
-                                      (130, 2048, "student_t"), (9, 8192, "outliers"), (3, 16384, "normal")])
+                                      (130, 2048, "student_t"), (9, 8192, "outliers"), (3, 16384, "normal"),
+                                      (1, 32, "normal"), (33, 2080, "student_t"), (2, 32768, "student_t")])
 @pytest.mark.parametrize("rounding", [ops.RNE, ops.SR])
 def test_nvfp4_forward(T, D, kind, rounding):
     x = _dev(synthetic.activations(T, D, kind, seed=T + 2 * D))
