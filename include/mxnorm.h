@@ -83,8 +83,9 @@ enum mxn_scale_layout {
     MXN_SCALES_MMA = 1
 };
 
-/* Bytes the scales of a [T, D] tensor occupy in the given layout; 0 if the
-   arguments are invalid. */
+/* Bytes the MX scales (one per 32 elements) of a [T, D] tensor occupy in the
+   given layout; 0 if the arguments are invalid.  NVFP4 scales are T * D / 16
+   bytes, row-major (MXN_ELEM_NVFP4 below). */
 size_t mxnorm_scales_bytes(int64_t T, int64_t D, int layout);
 
 /* Element format of the MX codes. */
