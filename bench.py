@@ -487,6 +487,18 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
                                "cores": oracle.num_threads(), "kind": "oracle",
                                "sample": f"all {T} rows of the workload, {passes} passes "
                                          f"({passes * dt:.1f} s, {dt * 1e3:.1f} ms per pass)"}
+        # and on one core: every (T / 256)-th row, repeated for about 2 s
+        rows1 = list(range(0, T, max(1, T // 256)))[:256]
+        passes1, t = 0, time.time()
+        while True:
+            oracle.mxnorm_fwd(x_cpu, g_cpu, p, rows=rows1, nthreads=1)
+            passes1 += 1
+            if time.time() - t >= 2.0:
+                break
+        dt1 = (time.time() - t) / passes1
+        out["cpu_baseline"]["value_1core"] = round(algorithmic_bytes(len(rows1), D) / dt1 / 1e9, 4)
+        out["cpu_baseline"]["sample_1core"] = (f"{len(rows1)} rows (one in {max(1, T // 256)}), 1 thread, "
+                                               f"{passes1} passes ({passes1 * dt1:.1f} s)")
     return out
 
 
