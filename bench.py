@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MXNorm fwd GB/s & % HBM peak at d=4096, vs RMSNorm+MXCast two-pass"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 7700.0          # B200 HBM3e, HGX datasheet figure
 
 
 def parse_args():
@@ -267,6 +268,7 @@ def run_ours(args, rank, world, local_rank):
         },
         "tokens_per_s": round(world * T / (ms_per_step * 1e-3), 1),
         "pct_hbm_peak": round(100.0 * value / (world * peak), 2),
+        "pct_hbm_nominal": round(100.0 * value / (world * NOMINAL_HBM_GBS), 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": profiled_traffic(args.workload),
                      "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json hbm_gbs' if peak_src == 'measured' else 'recipe fallback'})",
