@@ -242,12 +242,16 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int
   // Defaults measured on B200 with whole input and output sets rotating
   // through HBM (T = 8192 and 16384): one stage per group, and 512 threads
   // per CTA for rows of 33..64 blocks and of more than 256, 384 for 65..256
-  // blocks (12 one-warp rows or 6 two-warp rows in flight per SM).  Rows under
-  // 33 blocks, and stochastic rounding (bound by the Philox arithmetic, so it
-  // wants every warp the registers allow), keep the largest CTA with extra
-  // stages while 176 KB covers them.
+  // blocks of E4M3 codes (12 one-warp rows or 6 two-warp rows in flight per
+  // SM).  The FP4 formats do more arithmetic per byte and want the warps:
+  // 512 threads there too (MXFP4 / NVFP4 at 16384 x 8192: 65.5 -> 57.8 and
+  // 100.1 -> 85.6 us; at 8192 x 4096: 17.8 -> 17.4 and 27.2 -> 26.0 us).
+  // Rows under 33 blocks, and stochastic rounding (bound by the Philox
+  // arithmetic, so it wants every warp the registers allow), keep the largest
+  // CTA with extra stages while 176 KB covers them.
   const bool widest = bpt == 1 || sr;
-  const int def_threads = widest ? fwd_max_threads(bpt) : (bpt == 2 || C.tpr > 64 ? 512 : 384);
+  const bool fp4 = elem != kElemE4M3;
+  const int def_threads = widest ? fwd_max_threads(bpt) : (bpt == 2 || C.tpr > 64 || fp4 ? 512 : 384);
   if (g_tuning.stages) {
     C.stages = g_tuning.stages;
   } else if (widest) {
