@@ -200,3 +200,14 @@ def test_binding_checks_output_buffers(L):
     with pytest.raises(ValueError):
         _check_buffer([0] * 10, "q", 8, torch.uint8, cuda0)                            # not a tensor
     _check_buffer(None, "q", 8, torch.uint8, cuda0)                                     # allocated by the binding
+
+
+def test_binding_raises_when_the_library_is_missing(monkeypatch, tmp_path):
+    """No fallback: with the library file absent every op raises before doing work."""
+    import torch
+    monkeypatch.setattr(ops, "_lib", None)
+    monkeypatch.setattr(ops._build, "LIB", str(tmp_path / "libmxnorm_b200.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        ops.lib()
+    with pytest.raises((RuntimeError, ValueError)):      # refused, never computed on the host
+        ops.mxnorm_fwd(torch.zeros(2, 64, dtype=torch.bfloat16))
