@@ -10,7 +10,6 @@ other test already run.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
