@@ -261,7 +261,11 @@ int mxfp8_gemm(const void* a_q, const void* a_s, const void* b_q, const void* b_
  *
  * Same arguments, results and limits as mxnorm_bwd (D <= 16384), except that
  * the dgamma partial sums live in one 8 MiB scratch array inside this library
- * (2^21 fp32, allocated when a device loads the library, held until exit).
+ * (2^21 fp32).  The CUDA runtime reserves it on a device when the library's
+ * kernels are first used there (lazy module loading: not necessarily when the
+ * library is loaded), whether or not this entry point is ever called, and it
+ * stays until the process exits -- so every process that uses the library,
+ * each rank of a multi-GPU job included, holds 8 MiB on each device it uses.
  * The call allocates nothing.  To fit the scratch it may launch fewer CTAs
  * than mxnorm_bwd (every active row group writes its partial rows of D fp32,
  * at most 2^21 / D rows in all); it returns MXN_ERR_UNSUPPORTED if even one

@@ -264,10 +264,16 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int
   // gamma in shared memory: fp32 for up to 64 threads per row (D <= 8192), else bf16
   C.gamma_bytes = gamma_smem ? (uint32_t)align_up((gamma_fp32(C.tpr) ? 4u : 2u) * (uint32_t)D, 128) : 0u;
   const size_t per_group = (size_t)C.stages * C.stage_bytes;
-  // Shared memory per group: its ring, its 2 * stages barriers and its two
-  // reduction slot arrays; plus gamma and 16 bytes of alignment once.
-  const size_t per_group_all = per_group + (size_t)2 * C.stages * sizeof(uint64_t) +
-                               (size_t)2 * kRedSlots * sizeof(float2);
+  // MXNorm and MXCast rows of several warps stage each row's codes in shared
+  // memory and write them with one bulk copy (D bytes of E4M3, half that of
+  // E2M1); see kFwdBulkStores.
+  C.code_row_bytes = elem == kElemE4M3 ? (uint32_t)D : (uint32_t)D / 2u;
+  C.ostage_bytes = (mode == kModeRMSNorm || C.tpr <= 32) ? 0u : (uint32_t)align_up((size_t)C.rps * C.code_row_bytes, 128);
+  // Shared memory per group: its ring, its code staging buffer, its 2 * stages
+  // barriers and its two reduction slot arrays; plus gamma and 16 bytes of
+  // alignment once.
+  const size_t per_group_base = per_group + (size_t)2 * C.stages * sizeof(uint64_t) +
+                                (size_t)2 * kRedSlots * sizeof(float2);
   int ng;
   if (g_tuning.consumer_threads) {
     ng = g_tuning.consumer_threads / C.gthreads;
@@ -275,20 +281,25 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int
     ng = def_threads / C.gthreads;
   }
   int ng_max = fwd_max_threads(bpt) / C.gthreads;
-  const size_t fixed = C.gamma_bytes + 16;
+  const size_t fixed = C.gamma_bytes + 16 + (elem == kElemNVFP4 ? 128u * sizeof(float) : 0u);
   const size_t smem_cap = 227u * 1024u;
-  if (fixed + per_group_all > smem_cap)
+  if (fixed + per_group_base > smem_cap)
     return fail(MXN_ERR_UNSUPPORTED, "row of %d elements does not fit in shared memory", D);
-  const int ng_fit = (int)((smem_cap - fixed) / per_group_all);
+  int ng_fit = (int)((smem_cap - fixed) / per_group_base);
   if (ng_fit < ng_max) ng_max = ng_fit;
   ng = ng < 1 ? 1 : (ng > ng_max ? ng_max : ng);
+  // The staging buffers must not cost row groups: where they would, codes are
+  // stored directly.
+  if (C.ostage_bytes && fixed + (size_t)ng * (per_group_base + C.ostage_bytes) > smem_cap) C.ostage_bytes = 0;
   if (C.tpr > 32 && ng > 15) ng = 15;  // named barriers 1..15
   C.ng = ng;
   C.n_row_blocks = (T + C.rps - 1) / C.rps;
   C.ring_off = C.gamma_bytes;
-  C.bar_off = (uint32_t)align_up(C.ring_off + (size_t)ng * per_group, 16);
+  C.out_off = (uint32_t)align_up(C.ring_off + (size_t)ng * per_group, 128);
+  C.bar_off = (uint32_t)align_up(C.out_off + (size_t)ng * C.ostage_bytes, 16);
   C.red_off = C.bar_off + (uint32_t)(ng * 2 * C.stages * sizeof(uint64_t));
-  P->smem = C.red_off + (size_t)ng * 2 * kRedSlots * sizeof(float2);
+  C.rcp_off = (uint32_t)(C.red_off + (size_t)ng * 2 * kRedSlots * sizeof(float2));
+  P->smem = C.rcp_off + (elem == kElemNVFP4 ? 128u * sizeof(float) : 0u);
   P->threads = ng * C.gthreads;
   P->kernel = fwd_kernel(mode, sr, gamma_smem, elem, bpt, C.tpr);
   if (!P->kernel) return fail(MXN_ERR_UNSUPPORTED, "no kernel for D = %d", D);
@@ -320,7 +331,8 @@ int launch_fwd(int mode, bool sr, const FwdArgs& A, int64_t T, int D, int64_t ld
   if (rc) return rc;
   FwdArgs a = A;
   a.status = dev.status;
-  a.inv_K = 1.0f / (float)(A.elem == kElemNVFP4 ? D / 16 : D / kBlock);   // statistic blocks per row
+  a.n_stat = A.elem == kElemNVFP4 ? D / 16 : D / kBlock;   // statistic blocks per row
+  a.inv_n_stat = 1.0 / (double)a.n_stat;
   void* argv[] = {&a, &P.C};
   return launch_pdl(P.kernel, P.grid, P.threads, P.smem, argv, stream, "row_fwd_kernel launch");
 }
@@ -441,8 +453,9 @@ int launch_bwd(const BwdPlan& P, const BwdArgs& A, uint16_t* dgamma, cudaStream_
 // ----------------------------------------------- allocation-free backward
 //
 // Scratch for mxnorm_bwd_noalloc: the per-row-group dgamma partial sums, 2^21 fp32
-// (8 MiB).  Every device that loads this library holds it until the process
-// exits.  In host code the name is only a host-side stand-in; its device
+// (8 MiB).  The runtime reserves it on a device when the library's kernels are
+// first used there (whether or not mxnorm_bwd_noalloc is called) and holds it
+// until the process exits.  In host code the name is only a host-side stand-in; its device
 // address comes from cudaGetSymbolAddress, looked up once per device with
 // that device current.
 constexpr size_t kNoAllocScratchFloats = size_t(1) << 21;
@@ -522,7 +535,6 @@ static int fwd_like(int mode, const void* x, const void* gamma, void* q, void* s
   A.scales = static_cast<uint8_t*>(scales);
   A.G_out = G_out;
   A.p = p;
-  A.inv_p = std::isinf(p) ? 0.0f : 1.0f / p;
   A.pmode = pmode_of(p);
   A.seed_lo = (uint32_t)seed;
   A.seed_hi = (uint32_t)(seed >> 32);

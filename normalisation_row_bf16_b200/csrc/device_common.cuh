@@ -119,6 +119,34 @@ __device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gmem_s
       : "memory");
 }
 
+// 1-D bulk copy shared -> global on the TMA engine, tracked by the issuing
+// thread's bulk groups.  Needs 16-byte aligned addresses and a size that is a
+// multiple of 16.
+__device__ __forceinline__ void bulk_copy_s2g(void* gmem_dst, uint32_t smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
+               "r"(smem_src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed shared -> global copy of this thread has read its
+// source (the buffer may be rewritten) ...
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// ... or has completed its writes.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Order this thread's shared-memory writes before later bulk copies that read them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t a) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
+}
+
 // L2 policy for data read exactly once: evict first.
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
@@ -393,14 +421,17 @@ __device__ __forceinline__ void philox4x32_10_x2(uint4& a, uint4& b, const Philo
 // 2^-9, rare after the block scale) the same quantities in fp32: lo a multiple
 // of 2^-9, |v| - lo exact, the scaling by 2^41 a power of two; for an integer
 // r, r < t holds iff r < ceil(t), and ceil(t) < 2^32.
+//
+// The comparison needs no compare: with L the 20 dropped bits and r' = r >> 12,
+// r < L * 2^12 holds iff r' < L, iff L + (2^20 - 1 - r') >= 2^20, and
+// 2^20 - 1 - r' is (~r) >> 12.  So adding (~r) >> 12 to the bits of v carries
+// into the kept mantissa exactly when v rounds up (the carry may step into the
+// next binade, which is lo + step; it cannot reach the sign, |v| <= 448), and
+// clearing the 20 low bits leaves the grid value with v's sign.
 __device__ __forceinline__ float sr_e4m3_grid(float v, uint32_t r) {
   const uint32_t b = __float_as_uint(v);
   const uint32_t ab = b & 0x7FFFFFFFu;
-  if (ab >= 0x3C800000u) {
-    const uint32_t low = ab & 0xFFFFFu;
-    const uint32_t up = (r < (low << 12)) ? 0x100000u : 0u;
-    return __uint_as_float(((ab & 0xFFF00000u) + up) | (b & 0x80000000u));
-  }
+  if (ab >= 0x3C800000u) return __uint_as_float((b + ((~r) >> 12)) & 0xFFF00000u);
   const float a = __uint_as_float(ab);
   const float lo = truncf(a * 512.0f) * (1.0f / 512.0f);
   const uint32_t thr = __float2uint_ru((a - lo) * 2199023255552.0f);   // 2^41

@@ -14,8 +14,8 @@ import oracle
 from normalisation_row_bf16_b200 import build as nbuild
 from normalisation_row_bf16_b200 import ops, synthetic
 
-from parity_util import (BWD_RTOL_L2, bf16_ulp_distance, check_cast, check_mxnorm_fwd,
-                         mma_scale_offset, rel_l2, round_bf16, to_np_u8)
+from parity_util import (BWD_RTOL_L2, bf16_ulp_distance, check_bwd_elementwise, check_cast,
+                         check_mxnorm_fwd, mma_scale_offset, rel_l2, round_bf16, to_np_u8)
 
 pytestmark = pytest.mark.gpu
 
@@ -80,7 +80,7 @@ def test_mxnorm_fwd_sr_bit_exact(p):
     for seed in (0, 0x1234_5678_9ABC_DEF0):
         q, s, G = ops.mxnorm_fwd(xd, gd, p, rounding=ops.SR, seed=seed)
         torch.cuda.synchronize()
-        check_mxnorm_fwd(xd, gd, p, 1, seed, q, s, G, strict=False)
+        check_mxnorm_fwd(xd, gd, p, 1, seed, q, s, G)
 
 
 @pytest.mark.parametrize("T,D", [(1, 32), (3, 96), (5, 160), (64, 64), (130, 544), (257, 1056), (33, 2080),
@@ -94,7 +94,7 @@ def test_mxnorm_fwd_sr_ragged(T, D):
     xd, gd = _dev(x), _dev(g)
     q, s, G = ops.mxnorm_fwd(xd, gd, 2.0, rounding=ops.SR, seed=D)
     torch.cuda.synchronize()
-    check_mxnorm_fwd(xd, gd, 2.0, ops.SR, D, q, s, G, strict=False)
+    check_mxnorm_fwd(xd, gd, 2.0, ops.SR, D, q, s, G)
 
 
 def test_mxnorm_fwd_special_rows():
@@ -212,8 +212,10 @@ def test_mxnorm_bwd(T, D, with_gamma):
     torch.cuda.synchronize()
     dx_ref, dg_ref = oracle.mxnorm_bwd(x.cpu(), dy.cpu(), None if g is None else g.cpu(), G.cpu().numpy())
     assert rel_l2(dx.float().cpu().numpy(), round_bf16(dx_ref)) <= BWD_RTOL_L2
+    check_bwd_elementwise(dx, dx_ref, 1)
     if with_gamma:
         assert rel_l2(dg.float().cpu().numpy(), round_bf16(dg_ref)) <= BWD_RTOL_L2
+        check_bwd_elementwise(dg, dg_ref, None)
         # deterministic: a second call gives the same bits
         _, dg2 = ops.mxnorm_bwd(x, dy, g, G)
         assert torch.equal(dg, dg2)
@@ -249,7 +251,7 @@ def test_sweep_sampled_rows(D):
         for rounding in (ops.RNE, ops.SR):
             q, s, G = ops.mxnorm_fwd(x, None, p, rounding=rounding, seed=0)
             torch.cuda.synchronize()
-            check_mxnorm_fwd(x, None, p, rounding, 0, q, s, G, rows=rows, strict=False)
+            check_mxnorm_fwd(x, None, p, rounding, 0, q, s, G, rows=rows)
     del x
     torch.cuda.empty_cache()
 
@@ -265,8 +267,10 @@ def test_bwd_full_size_sampled():
     rows = _sample_rows(T)
     dx_ref, _ = oracle.mxnorm_bwd(x.cpu(), dy.cpu(), g.cpu(), G.cpu().numpy()[rows], rows=rows)
     assert rel_l2(dx.float().cpu().numpy()[rows], round_bf16(dx_ref)) <= BWD_RTOL_L2
+    check_bwd_elementwise(dx.cpu()[torch.from_numpy(rows)], dx_ref, 1)
     _, dg_ref = oracle.mxnorm_bwd(x.cpu(), dy.cpu(), g.cpu(), G.cpu().numpy())
     assert rel_l2(dg.float().cpu().numpy(), round_bf16(dg_ref)) <= BWD_RTOL_L2
+    check_bwd_elementwise(dg, dg_ref, None)
 
 
 def test_tuning_variants_agree():
@@ -303,7 +307,7 @@ def test_more_than_2_31_elements_sampled_rows():
     for rounding in (ops.RNE, ops.SR):
         q, s, G = ops.mxnorm_fwd(x, g, 2.0, rounding=rounding, seed=11)
         torch.cuda.synchronize()
-        check_mxnorm_fwd(x, g, 2.0, rounding, 11, q, s, G, rows=rows, strict=False)
+        check_mxnorm_fwd(x, g, 2.0, rounding, 11, q, s, G, rows=rows)
         del q, s, G
         torch.cuda.empty_cache()
     dy = synthetic.upstream_grad(T, D, seed=3, device="cuda")
@@ -313,6 +317,7 @@ def test_more_than_2_31_elements_sampled_rows():
     sel = torch.from_numpy(rows).cuda()
     dx_ref, _ = oracle.mxnorm_bwd(x[sel].cpu(), dy[sel].cpu(), g.cpu(), G[sel].cpu().numpy())
     assert rel_l2(dx[sel].double().cpu().numpy(), round_bf16(dx_ref)) <= BWD_RTOL_L2
+    check_bwd_elementwise(dx[sel], dx_ref, 1)
     assert torch.isfinite(dg.float()).all()
     del x, dy, dx, G
     torch.cuda.empty_cache()

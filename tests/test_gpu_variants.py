@@ -226,11 +226,11 @@ def test_variants_llama8b_shape_sampled_rows(elem, stat):
     torch.cuda.synchronize()
     rows = np.concatenate([np.arange(0, 8), np.random.default_rng(2).choice(w["T"], 40, replace=False),
                            np.arange(w["T"] - 8, w["T"])])
-    check_mxnorm_fwd(x, g, 2.0, ops.RNE, 0, q, s, G, rows=rows, strict=False, stat=stat, fmt=elem)
+    check_mxnorm_fwd(x, g, 2.0, ops.RNE, 0, q, s, G, rows=rows, stat=stat, fmt=elem)
     for rnd in (ops.SR,):
         q, s, G = ops.mxnorm_fwd_ex(x, g, 2.0, rounding=rnd, seed=5, elem=elem, stat=stat)
         torch.cuda.synchronize()
-        check_mxnorm_fwd(x, g, 2.0, rnd, 5, q, s, G, rows=rows[:16], strict=False, stat=stat, fmt=elem)
+        check_mxnorm_fwd(x, g, 2.0, rnd, 5, q, s, G, rows=rows[:16], stat=stat, fmt=elem)
 
 
 def test_fold_weight_full_qkv_sampled_rows():
@@ -366,7 +366,7 @@ def test_nvfp4_llama8b_shape_sampled_rows():
     for rnd in (ops.RNE, ops.SR):
         q, s, G = ops.mxnorm_fwd_ex(x, g, 2.0, rounding=rnd, seed=2, elem="nvfp4")
         torch.cuda.synchronize()
-        check_mxnorm_fwd(x, g, 2.0, rnd, 2, q, s, G, rows=rows, strict=False, fmt="nvfp4")
+        check_mxnorm_fwd(x, g, 2.0, rnd, 2, q, s, G, rows=rows, fmt="nvfp4")
 
 
 def test_binding_rejects_undersized_outputs():
