@@ -46,8 +46,8 @@ def parse_args():
     ap.add_argument("--workload", default="llama8b_8192x4096_outliers_p2")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the two-pass comparator, e2e and CPU baseline legs")
-    ap.add_argument("--sweep", action="store_true",
-                    help="also time MXNorm forward over the sweep shapes (16384 x {2048..16384}, p in {1,2,4,inf}, RNE/SR)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the sweep legs (16384 x {2048..16384}, p in {1,2,4,inf}, RNE/SR)")
     ap.add_argument("--soak-s", type=float, default=0.5,
                     help="untimed back-to-back steps before timing, so clocks settle under load")
     ap.add_argument("--profile-only", choices=["fwd", "sr", "mxfp4", "nvfp4", "bwd", "gemm"], default=None,
@@ -95,23 +95,86 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", f"mxnorm_fwd_{workload}.md")
+def profile_fields(name):
+    """The "- key: value" fields of a committed ncu summary under profiles/, if
+    it was taken on the current kernel sources (else {})."""
+    path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
-        return None
+        return {}
     fields = {}
     for line in open(path):
         if line.startswith("- ") and ":" in line:
             k, v = line[2:].split(":", 1)
             fields[k.strip()] = v.strip().strip("`")
     if fields.get("kernel_source_hash") != kernel_source_hash():
-        return None
+        return {}
+    return fields
+
+
+def _int_field(fields, key):
     try:
-        return int(fields["dram_bytes_per_launch"])
+        return int(fields[key])
     except (KeyError, ValueError):
         return None
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch (steady state: the mean over captured launches that
+    follow other launches) from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    return _int_field(profile_fields(f"mxnorm_fwd_{workload}.md"), "dram_bytes_per_launch")
+
+
+def profiled_traffic_split(workload):
+    f = profile_fields(f"mxnorm_fwd_{workload}.md")
+    r, w = _int_field(f, "dram_read_bytes_per_launch"), _int_field(f, "dram_write_bytes_per_launch")
+    return None if r is None or w is None else {"read": r, "write": w}
+
+
+def profiled_instructions(name, key):
+    """Thread instructions per element of a kernel from a committed ncu summary
+    (current sources only), else None."""
+    try:
+        return float(profile_fields(name)[key])
+    except (KeyError, ValueError):
+        return None
+
+
+def issue_peak(sm_mhz):
+    """Lane-instructions per second the SMs can issue: 148 SMs x 4 schedulers x
+    one warp-instruction (32 lanes) per clock, at the sampled SM clock."""
+    return 148 * 4 * 32 * sm_mhz * 1e6
+
+
+def alu_roofline(instr_per_elem, elements, ms, sm_mhz):
+    """Issue-rate roofline of a launch: thread instructions per element (from
+    the committed ncu summary of the same kernel and workload) times the
+    elements, over the launch time, against the issue peak at the sampled SM
+    clock.  None when either figure is missing."""
+    if not instr_per_elem or not sm_mhz:
+        return None
+    achieved = instr_per_elem * elements / (ms * 1e-3)
+    peak = issue_peak(sm_mhz)
+    return {"bound": "alu", "instr_per_elem": round(instr_per_elem, 2), "achieved_Tinstr_s": round(achieved / 1e12, 2),
+            "peak_Tinstr_s": round(peak / 1e12, 2), "frac": round(achieved / peak, 4), "sm_mhz": sm_mhz}
+
+
+def compact(leg, extra=None):
+    """A graph leg's record as the bench line carries it: time per launch,
+    GB/s of algorithmic bytes and the fraction of the HBM peak."""
+    out = {"us": round(leg["ms"] * 1e3, 2), "GBps": leg["GBps"], "frac": leg["roofline"]["frac"]}
+    if extra:
+        out.update(extra)
+    return out
+
+
+def device_hold():
+    """Queue a short spin kernel (torch's, about 0.25 ms) ahead of a timed
+    region's start event.  The device is then busy while the host enqueues the
+    start event and the graph, so the region starts when the device reaches it
+    and the first step does not include the host's graph-launch latency."""
+    import torch
+    torch.cuda._sleep(500_000)
 
 
 class ClockSampler:
@@ -229,6 +292,7 @@ def run_ours(args, rank, world, local_rank):
     graph.replay()                     # untimed: first replay uploads the graph
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
+    device_hold()
     t0.record()
     graph.replay()
     t1.record()
@@ -246,42 +310,59 @@ def run_ours(args, rank, world, local_rank):
 
     extras = {}
     if not args.no_extras:
-        extras = run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step)
+        sm_mhz = (clocks or {}).get("sm_mhz") if rank == 0 else None
+        extras = run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step, sm_mhz)
 
     if rank != 0:
         return None
     peaks, peak_src = measured_peaks()
     achieved = nbytes / (mean_kern_ms * 1e-3) / 1e9
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": profiled_traffic(args.workload),
+            "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json hbm_gbs' if peak_src == 'measured' else 'recipe fallback'})",
+            "algorithmic_bytes_per_launch": nbytes,
+            "kernel": "row_fwd_kernel<MXNorm>", "mean_launch_ms": round(mean_kern_ms, 6)}
+    split = profiled_traffic_split(args.workload)
+    if split:
+        roof["traffic_read"], roof["traffic_write"] = split["read"], split["write"]
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {
             "workload": args.workload, "T": T, "D": D, "block": 32, "p": p, "rounding": "rne",
-            "timing": "K steps captured in one CUDA graph, replayed between CUDA events",
+            "timing": "K steps captured in one CUDA graph, replayed between CUDA events "
+                      "(a spin kernel queued ahead of the start event keeps the graph-launch latency out)",
             "gamma": True, "scale_layout": "rowmajor", "x": w["kind"],
             "l2": f"inputs rotate over {n_sets} sets of {set_bytes / 2**20:.0f} MiB "
                   f"({n_sets * set_bytes / 2**20:.0f} MiB > 3x the 126 MB L2)",
             "parallelism": f"replicas x{world}: each rank its own {T}-row batch, no collective",
             "clock_soak_s": args.soak_s,
         },
-        "tokens_per_s": round(world * T / (ms_per_step * 1e-3), 1),
-        "pct_hbm_peak": round(100.0 * value / (world * peak), 2),
-        "pct_hbm_nominal": round(100.0 * value / (world * NOMINAL_HBM_GBS), 2),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(args.workload),
-                     "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json hbm_gbs' if peak_src == 'measured' else 'recipe fallback'})",
-                     "algorithmic_bytes_per_launch": nbytes,
-                     "kernel": "row_fwd_kernel<MXNorm>", "mean_launch_ms": round(mean_kern_ms, 6)},
+        "roofline": roof,
         "gpu_launches": K,
         "clocks": clocks,
     }
+    # Bulky context first, the figures the summary reads last (a reader of the
+    # line's tail sees them).
+    order = ["cpu_baseline", "e2e", "stream_context", "gemm", "fold_weight", "pipeline_mxnorm_gemm",
+             "pipeline_rmsnorm_mxcast_gemm", "pipeline_speedup", "mxfp4_fwd", "nvfp4_fwd", "scale_reuse_fwd",
+             "sweep", "tiny", "bwd", "sr_fwd", "parity"]
+    for k in order:
+        if k in extras:
+            line[k] = extras.pop(k)
     line.update(extras)
+    line["tokens_per_s"] = round(world * T / (ms_per_step * 1e-3), 1)
+    line["pct_hbm_nominal"] = round(100.0 * value / (world * NOMINAL_HBM_GBS), 2)
+    line["pct_hbm_peak"] = round(100.0 * value / (world * peak), 2)
+    for k in ("two_pass", "speedup_vs_two_pass"):
+        if k in line:
+            line[k] = line.pop(k)
     return line
 
 
-def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
+def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step, sm_mhz):
     """Two-pass comparator, end-to-end through host buffers, CPU oracle."""
     import torch
     import torch.distributed as dist
@@ -310,6 +391,7 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
     g2.replay()
     barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    device_hold()
     t0.record()
     g2.replay()
     t1.record()
@@ -392,21 +474,29 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
     # Every leg rotates whole input and output sets (> 3x L2), like the headline.
     outs = [(torch.empty(T, D, dtype=torch.uint8, device=dev), torch.empty(T, D // 32, dtype=torch.uint8, device=dev),
              torch.empty(T, dtype=torch.float32, device=dev)) for _ in range(n_sets)]
-    out["sr_fwd"] = run_graph_leg(args, world, dev, barrier,
-                                  lambda i: ops.mxnorm_fwd(xs[i % n_sets], g, p, rounding=ops.SR, seed=i,
-                                                           q=outs[i % n_sets][0], scales=outs[i % n_sets][1],
-                                                           G=outs[i % n_sets][2]),
-                                  algorithmic_bytes(T, D), "row_fwd_kernel<MXNorm, SR>")
+    sr = run_graph_leg(args, world, dev, barrier,
+                       lambda i: ops.mxnorm_fwd(xs[i % n_sets], g, p, rounding=ops.SR, seed=i,
+                                                q=outs[i % n_sets][0], scales=outs[i % n_sets][1],
+                                                G=outs[i % n_sets][2]),
+                       algorithmic_bytes(T, D), "row_fwd_kernel<MXNorm, SR>")
+    out["sr_fwd"] = compact(sr, {"alu": alu_roofline(
+        profiled_instructions(f"mxnorm_fwd_sr_{args.workload}.md", "thread_instructions_per_element"),
+        T * D, sr["ms"], sm_mhz)})
     del outs
     dys = [synthetic.upstream_grad(T, D, seed=j, device=dev) for j in range(n_sets)]
     dxs = [torch.empty_like(xs[0]) for _ in range(n_sets)]
     Gbs = [ops.mxnorm_fwd(xs[j], g, p)[2] for j in range(n_sets)]
     dgb = torch.empty(D, dtype=torch.bfloat16, device=dev)
     wsb = torch.empty(max(16, ops.bwd_workspace_bytes(T, D)), dtype=torch.uint8, device=dev)
-    out["bwd"] = run_graph_leg(args, world, dev, barrier,
-                               lambda i: ops.mxnorm_bwd(xs[i % n_sets], dys[i % n_sets], g, Gbs[i % n_sets],
-                                                        dx=dxs[i % n_sets], dgamma=dgb, workspace=wsb),
-                               bwd_bytes(T, D, wsb.numel()), "row_bwd_kernel + dgamma_reduce_kernel")
+    bw = run_graph_leg(args, world, dev, barrier,
+                       lambda i: ops.mxnorm_bwd(xs[i % n_sets], dys[i % n_sets], g, Gbs[i % n_sets],
+                                                dx=dxs[i % n_sets], dgamma=dgb, workspace=wsb),
+                       bwd_bytes(T, D, 0), "row_bwd_kernel + dgamma_reduce_kernel")
+    # frac counts the algorithmic bytes (x, dy, dx, G, gamma, dgamma); the dgamma
+    # partial rows written and read back are traffic on top, shown apart
+    ws = ops.bwd_workspace_bytes(T, D)
+    out["bwd"] = compact(bw, {"workspace_bytes": 2 * ws,
+                              "GBps_with_workspace": round(world * bwd_bytes(T, D, ws) / (bw["ms"] * 1e-3) / 1e9, 1)})
     del dys, dxs, Gbs
 
     # Size context for the headline's roofline fraction: the measured HBM peak
@@ -428,16 +518,16 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
                                              lambda i: f8s[i % n_sets].copy_(xs[i % n_sets]), 3 * T * D,
                                              "torch elementwise cast bf16 -> float8_e4m3fn of x (no scales)")
     del f8s
-    for v in ctx.values():
-        v["headline_over_this"] = round(v["ms"] / ms_per_step * algorithmic_bytes(T, D) / v["roofline"]
-                                        ["algorithmic_bytes_per_launch"], 3)
-    out["stream_context"] = ctx
+    out["stream_context"] = {
+        k: compact(v, {"headline_over_this": round(v["ms"] / ms_per_step * algorithmic_bytes(T, D) /
+                                                   v["roofline"]["algorithmic_bytes_per_launch"], 3)})
+        for k, v in ctx.items()}
 
     # Variants on the same batch: MXFP4 codes, the scale-reuse statistic.
     outs4 = [(torch.empty(T, D // 2, dtype=torch.uint8, device=dev),
               torch.empty(T, D // 32, dtype=torch.uint8, device=dev),
               torch.empty(T, dtype=torch.float32, device=dev)) for _ in range(n_sets)]
-    out["mxfp4_fwd"] = run_graph_leg(args, world, dev, barrier,
+    out["mxfp4_fwd"] = compact_leg(args, world, dev, barrier,
                                      lambda i: ops.mxnorm_fwd_ex(xs[i % n_sets], g, p, elem="e2m1",
                                                                  q=outs4[i % n_sets][0], scales=outs4[i % n_sets][1],
                                                                  G=outs4[i % n_sets][2]),
@@ -446,7 +536,7 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
     outsn = [(torch.empty(T, D // 2, dtype=torch.uint8, device=dev),
               torch.empty(T, D // 16, dtype=torch.uint8, device=dev),
               torch.empty(T, dtype=torch.float32, device=dev)) for _ in range(n_sets)]
-    out["nvfp4_fwd"] = run_graph_leg(args, world, dev, barrier,
+    out["nvfp4_fwd"] = compact_leg(args, world, dev, barrier,
                                      lambda i: ops.mxnorm_fwd_ex(xs[i % n_sets], g, p, elem="nvfp4",
                                                                  q=outsn[i % n_sets][0], scales=outsn[i % n_sets][1],
                                                                  G=outsn[i % n_sets][2]),
@@ -454,7 +544,7 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
     del outsn
     outs = [(torch.empty(T, D, dtype=torch.uint8, device=dev), torch.empty(T, D // 32, dtype=torch.uint8, device=dev),
              torch.empty(T, dtype=torch.float32, device=dev)) for _ in range(n_sets)]
-    out["scale_reuse_fwd"] = run_graph_leg(args, world, dev, barrier,
+    out["scale_reuse_fwd"] = compact_leg(args, world, dev, barrier,
                                            lambda i: ops.mxnorm_fwd_ex(xs[i % n_sets], g, p, stat="scale_exp",
                                                                        q=outs[i % n_sets][0], scales=outs[i % n_sets][1],
                                                                        G=outs[i % n_sets][2]),
@@ -468,8 +558,9 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
         out["gemm"] = run_gemm_leg(args, w, rank, world, dev, barrier)
         out.update(run_linear_legs(args, w, rank, world, dev, barrier))
 
-    if args.sweep:
-        out["sweep"] = run_sweep(args, world, dev, barrier)
+    if not args.no_sweep:
+        out["sweep"] = run_sweep(args, world, dev, barrier, sm_mhz)
+    out["tiny"] = run_tiny(args, world, dev, barrier)
 
     # CPU oracle on the host cores: rank 0, one GPU only
     if rank == 0 and world == 1:
@@ -479,12 +570,30 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
         oracle.mxnorm_fwd(x_cpu[:64], g_cpu, p)             # load + warm
         # whole passes over the workload until about 10 s of CPU work
         passes, t = 0, time.time()
+        first = None
         while True:
-            oracle.mxnorm_fwd(x_cpu, g_cpu, p)
+            res = oracle.mxnorm_fwd(x_cpu, g_cpu, p)
+            first = res if first is None else first
             passes += 1
             if time.time() - t >= 10.0:
                 break
         dt = (time.time() - t) / passes
+        # The oracle's pass above is the reference for the GPU's result on the
+        # same batch (one more launch, after every timed region): counts of G
+        # bits, E8M0 scales and E4M3 codes that differ from the oracle's own.
+        q_o, s_o, G_o = first
+        q_g, s_g, G_g = ops.mxnorm_fwd(xs[0], g, p)
+        torch.cuda.synchronize()
+        q_g = q_g.cpu().numpy()
+        s_g = s_g.cpu().numpy()
+        G_g = G_g.cpu().numpy()
+        import numpy as np
+        rel = np.abs(G_g.astype(np.float64) - G_o.astype(np.float64)) / np.maximum(G_o.astype(np.float64), 1e-300)
+        out["parity"] = {"vs": "oracle's own result, every row of the batch", "rows": int(T),
+                         "G_bit_mismatch_rows": int(np.count_nonzero(G_g.view(np.uint32) != G_o.view(np.uint32))),
+                         "G_max_rel": float(rel.max()),
+                         "scale_mismatch": int(np.count_nonzero(s_g != s_o)),
+                         "code_mismatch": int(np.count_nonzero(q_g != q_o))}
         out["cpu_baseline"] = {"value": round(algorithmic_bytes(T, D) / dt / 1e9, 3), "unit": "GB/s",
                                "cores": oracle.num_threads(), "kind": "oracle",
                                "sample": f"all {T} rows of the workload, {passes} passes "
@@ -502,6 +611,31 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step):
         out["cpu_baseline"]["sample_1core"] = (f"{len(rows1)} rows (one in {max(1, T // 256)}), 1 thread, "
                                                f"{passes1} passes ({passes1 * dt1:.1f} s)")
     return out
+
+
+def compact_leg(args, world, dev, barrier, fn, nbytes, kernel):
+    return compact(run_graph_leg(args, world, dev, barrier, fn, nbytes, kernel))
+
+
+def run_tiny(args, world, dev, barrier):
+    """The small configuration (x bf16 [256 x 1024] N(0,1), gamma, p = 2,
+    nearest-even): one launch moves 0.79 MB, so it is launch-bound; reported
+    for completeness."""
+    import torch
+    from normalisation_row_bf16_b200 import ops, synthetic
+    w = workload_cfg("tiny_256x1024_normal_p2")
+    T, D, p = w["T"], w["D"], w["p"]
+    x = synthetic.activations(T, D, w["kind"], seed=0, device=dev)
+    g = synthetic.gamma(D, seed=0, device=dev)
+    n = 8
+    xs = [x] + [x.clone() for _ in range(n - 1)]
+    outs = [(torch.empty(T, D, dtype=torch.uint8, device=dev), torch.empty(T, D // 32, dtype=torch.uint8, device=dev),
+             torch.empty(T, dtype=torch.float32, device=dev)) for _ in range(n)]
+    leg = run_graph_leg(args, world, dev, barrier,
+                        lambda i: ops.mxnorm_fwd(xs[i % n], g, p, q=outs[i % n][0], scales=outs[i % n][1],
+                                                 G=outs[i % n][2]),
+                        algorithmic_bytes(T, D), "row_fwd_kernel<MXNorm>")
+    return compact(leg, {"workload": "tiny_256x1024_normal_p2", "note": "launch-bound (0.79 MB per launch), L2-resident"})
 
 
 def bwd_bytes(T, D, ws_bytes):
@@ -524,6 +658,7 @@ def run_graph_leg(args, world, dev, barrier, fn, nbytes, kernel):
     graph.replay()
     barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    device_hold()
     t0.record()
     graph.replay()
     t1.record()
@@ -542,7 +677,12 @@ def run_graph_leg(args, world, dev, barrier, fn, nbytes, kernel):
             "kernel": kernel}
 
 
-def run_sweep(args, world, dev, barrier):
+def run_sweep(args, world, dev, barrier, sm_mhz):
+    """T = 16384, D in {2048, 4096, 8192, 16384}, x = 0.5 t(3), no gamma, p in
+    {1, 2, 4, inf}, nearest-even and stochastic rounding.  One compact record
+    per case: [D, p, rounding, us, GB/s, fraction of HBM, fraction of the issue
+    rate (stochastic rounding at p = 2, where a committed instruction count
+    exists)]."""
     import math as _m
     import torch
     from normalisation_row_bf16_b200 import ops, synthetic
@@ -558,6 +698,7 @@ def run_sweep(args, world, dev, barrier):
         qs = [torch.empty(T, D, dtype=torch.uint8, device=dev) for _ in range(n_rot)]
         scs = [torch.empty(T, D // 32, dtype=torch.uint8, device=dev) for _ in range(n_rot)]
         Gs = [torch.empty(T, dtype=torch.float32, device=dev) for _ in range(n_rot)]
+        ipe = profiled_instructions("mxnorm_fwd_sr_sweep_16384.md", f"thread_instructions_per_element_D{D}")
         for p in (1.0, 2.0, 4.0, _m.inf):
             for rnd in (ops.RNE, ops.SR):
                 r = run_graph_leg(args, world, dev, barrier,
@@ -565,12 +706,16 @@ def run_sweep(args, world, dev, barrier):
                                                            q=qs[i % n_rot], scales=scs[i % n_rot],
                                                            G=Gs[i % n_rot]),
                                   algorithmic_bytes(T, D) - 2 * D, "row_fwd_kernel<MXNorm>")
-                res.append({"T": T, "D": D, "p": "inf" if _m.isinf(p) else p,
-                            "rounding": "sr" if rnd == ops.SR else "rne", "ms": r["ms"],
-                            "GBps": r["GBps"], "frac": r["roofline"]["frac"]})
+                rec = [D, "inf" if _m.isinf(p) else int(p), "sr" if rnd == ops.SR else "rne",
+                       round(r["ms"] * 1e3, 1), round(r["GBps"]), round(r["roofline"]["frac"], 3)]
+                if rnd == ops.SR and p == 2.0:
+                    alu = alu_roofline(ipe, T * D, r["ms"], sm_mhz)
+                    rec.append(alu["frac"] if alu else None)
+                res.append(rec)
         del x, xs2, qs, scs, Gs
         torch.cuda.empty_cache()
-    return res
+    return {"T": 16384, "x": "0.5 t(3)", "gamma": False,
+            "fields": ["D", "p", "rounding", "us", "GBps", "frac_hbm", "frac_issue (sr, p=2)"], "cases": res}
 
 
 def run_gemm_leg(args, w, rank, world, dev, barrier):
@@ -595,6 +740,7 @@ def run_gemm_leg(args, w, rank, world, dev, barrier):
     graph.replay()
     barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    device_hold()
     t0.record()
     graph.replay()
     t1.record()
