@@ -50,8 +50,11 @@ def parse_args():
                     help="skip the sweep legs (16384 x {2048..16384}, p in {1,2,4,inf}, RNE/SR)")
     ap.add_argument("--soak-s", type=float, default=0.5,
                     help="untimed back-to-back steps before timing, so clocks settle under load")
-    ap.add_argument("--profile-only", choices=["fwd", "sr", "mxfp4", "nvfp4", "bwd", "gemm"], default=None,
-                    help="run only this kernel, 4 launches on the workload, untimed (for ncu captures)")
+    ap.add_argument("--profile-only", choices=["fwd", "sr", "mxfp4", "nvfp4", "bwd", "gemm", "sr_sweep"],
+                    default=None,
+                    help="run only this kernel, 8 launches on the workload with inputs and outputs "
+                         "rotating over 4 sets, untimed (for ncu captures); "
+                         "sr_sweep: two stochastic-rounding launches per sweep shape (T = 16384, p = 2)")
     return ap.parse_args()
 
 
@@ -875,35 +878,59 @@ def run_profile_only(args):
     batch; the GEMM on the fused QKV weight), for a profiler to capture."""
     import torch
     from normalisation_row_bf16_b200 import ops, synthetic
+    leg = args.profile_only
+    if leg == "sr_sweep":
+        for Ds in (2048, 4096, 8192, 16384):
+            xs = synthetic.activations(16384, Ds, "student_t", seed=1, device="cuda")
+            for i in range(2):
+                ops.mxnorm_fwd(xs, None, 2.0, rounding=ops.SR, seed=i)
+            torch.cuda.synchronize()
+            del xs
+            torch.cuda.empty_cache()
+        if ops.device_status() != ops.MXN_OK:
+            raise SystemExit("device status not clean")
+        print(json.dumps({"profile_only": leg, "launches": 8}), flush=True)
+        return
     w = workload_cfg(args.workload)
     T, D, p = w["T"], w["D"], w["p"]
     x = synthetic.activations(T, D, w.get("kind", "outliers"), seed=0, device="cuda")
     g = synthetic.gamma(D, seed=0, device="cuda")
-    leg = args.profile_only
+    # Inputs and outputs rotate over 4 sets (> 3x L2) as in the timed legs, so
+    # a captured launch sees the steady state's DRAM traffic: its inputs come
+    # from DRAM and the write-backs of earlier launches' outputs land in it.
+    n = 4
+    xs = [x] + [x.clone() for _ in range(n - 1)]
     if leg == "bwd":
-        dy = synthetic.upstream_grad(T, D, seed=0, device="cuda")
-        _, _, G = ops.mxnorm_fwd(x, g, p)
+        dys = [synthetic.upstream_grad(T, D, seed=j, device="cuda") for j in range(n)]
+        Gs = [ops.mxnorm_fwd(xs[j], g, p)[2] for j in range(n)]
+        dxs = [torch.empty_like(x) for _ in range(n)]
     if leg == "gemm":
         wt = synthetic.gemm_weight(6144, D, seed=0, device="cuda")
         aq, a_s, _ = ops.mxnorm_fwd(x, None, p, scale_layout=ops.SCALES_MMA)
         bq, b_s = ops.fold_weight(wt, g)
-    for i in range(4):
+    cw = D // 2 if leg in ("mxfp4", "nvfp4") else D
+    sw = D // 16 if leg == "nvfp4" else D // 32
+    outs = [(torch.empty(T, cw, dtype=torch.uint8, device="cuda"), torch.empty(T, sw, dtype=torch.uint8, device="cuda"),
+             torch.empty(T, dtype=torch.float32, device="cuda")) for _ in range(n)]
+    for i in range(8):
+        j = i % n
+        q, s, Gq = outs[j]
         if leg == "fwd":
-            ops.mxnorm_fwd(x, g, p)
+            ops.mxnorm_fwd(xs[j], g, p, q=q, scales=s, G=Gq)
         elif leg == "sr":
-            ops.mxnorm_fwd(x, g, p, rounding=ops.SR, seed=i)
+            ops.mxnorm_fwd(xs[j], g, p, rounding=ops.SR, seed=i, q=q, scales=s, G=Gq)
         elif leg == "mxfp4":
-            ops.mxnorm_fwd_ex(x, g, p, elem="e2m1")
+            ops.mxnorm_fwd_ex(xs[j], g, p, elem="e2m1", q=q, scales=s, G=Gq)
         elif leg == "nvfp4":
-            ops.mxnorm_fwd_ex(x, g, p, elem="nvfp4")
+            ops.mxnorm_fwd_ex(xs[j], g, p, elem="nvfp4", q=q, scales=s, G=Gq)
         elif leg == "bwd":
-            ops.mxnorm_bwd(x, dy, g, G)
+            ops.mxnorm_bwd(xs[j], dys[j], g, Gs[j], dx=dxs[j])
         elif leg == "gemm":
             ops.mxfp8_gemm(aq, a_s, bq, b_s, T, 6144, D)
     torch.cuda.synchronize()
     if ops.device_status() != ops.MXN_OK:
         raise SystemExit("device status not clean")
-    print(json.dumps({"profile_only": leg, "launches": 4}), flush=True)
+    print(json.dumps({"profile_only": leg, "launches": 8}), flush=True)
 
 
 def main():

@@ -268,7 +268,7 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int
   // memory and write them with one bulk copy (D bytes of E4M3, half that of
   // E2M1); see kFwdBulkStores.
   C.code_row_bytes = elem == kElemE4M3 ? (uint32_t)D : (uint32_t)D / 2u;
-  C.ostage_bytes = (mode == kModeRMSNorm || C.tpr <= 32) ? 0u : (uint32_t)align_up((size_t)C.rps * C.code_row_bytes, 128);
+  C.ostage_bytes = (mode == kModeRMSNorm || C.tpr <= 32 || sr) ? 0u : (uint32_t)align_up((size_t)C.rps * C.code_row_bytes, 128);
   // Shared memory per group: its ring, its code staging buffer, its 2 * stages
   // barriers and its two reduction slot arrays; plus gamma and 16 bytes of
   // alignment once.
@@ -280,7 +280,7 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int
   } else {
     ng = def_threads / C.gthreads;
   }
-  int ng_max = fwd_max_threads(bpt) / C.gthreads;
+  int ng_max = fwd_launch_threads(bpt, C.tpr, sr, elem) / C.gthreads;
   const size_t fixed = C.gamma_bytes + 16 + (elem == kElemNVFP4 ? 128u * sizeof(float) : 0u);
   const size_t smem_cap = 227u * 1024u;
   if (fixed + per_group_base > smem_cap)
@@ -333,6 +333,7 @@ int launch_fwd(int mode, bool sr, const FwdArgs& A, int64_t T, int D, int64_t ld
   a.status = dev.status;
   a.n_stat = A.elem == kElemNVFP4 ? D / 16 : D / kBlock;   // statistic blocks per row
   a.inv_n_stat = 1.0 / (double)a.n_stat;
+  a.inv_k_pow2 = (a.n_stat & (a.n_stat - 1)) == 0 ? (float)a.inv_n_stat : 0.0f;
   void* argv[] = {&a, &P.C};
   return launch_pdl(P.kernel, P.grid, P.threads, P.smem, argv, stream, "row_fwd_kernel launch");
 }
@@ -388,18 +389,28 @@ int plan_bwd(int64_t T, int D, int sms, BwdPlan* P, int64_t max_partial_rows = 0
   // 49.1 with two stages and 51.6 with three groups of two stages).
   const int stages = g_tuning.stages ? g_tuning.stages : 1;
   C.gamma_bytes = (uint32_t)align_up(2u * (uint32_t)D, 128);
+  // dx staged per group and written with one bulk copy per row block, while
+  // the buffers fit beside the rings of the planned groups.
+  C.ostage_bytes = (uint32_t)align_up((size_t)C.rps * C.row_bytes, 128);
   auto smem_of = [&](int n) {
     return (size_t)C.gamma_bytes + (size_t)n * stages * (C.stage_bytes + 2 * sizeof(uint64_t)) +
-           (size_t)n * per_group_fixed + 16;
+           (size_t)n * (per_group_fixed + C.ostage_bytes) + 128 + 16;
   };
-  while (ng > 1 && smem_of(ng) > smem_cap) --ng;
+  {
+    const uint32_t keep = C.ostage_bytes;
+    C.ostage_bytes = 0;
+    while (ng > 1 && smem_of(ng) > smem_cap) --ng;
+    C.ostage_bytes = keep;
+    if (smem_of(ng) > smem_cap) C.ostage_bytes = 0;
+  }
   if (smem_of(ng) > smem_cap)
     return fail(MXN_ERR_UNSUPPORTED, "mxnorm_bwd: a row of %d elements does not fit in shared memory", D);
   C.ng = ng;
   C.stages = stages;
   C.n_row_blocks = (T + C.rps - 1) / C.rps;
   C.ring_off = C.gamma_bytes;
-  C.bar_off = (uint32_t)align_up(C.ring_off + (size_t)ng * stages * C.stage_bytes, 16);
+  C.out_off = (uint32_t)align_up(C.ring_off + (size_t)ng * stages * C.stage_bytes, 128);
+  C.bar_off = (uint32_t)align_up(C.out_off + (size_t)ng * C.ostage_bytes, 16);
   C.red_off = C.bar_off + (uint32_t)(ng * 2 * stages * sizeof(uint64_t));
   P->smem = C.red_off + (size_t)ng * 2 * kRedSlots * sizeof(float2);
   P->threads = ng * C.gthreads;

@@ -49,6 +49,8 @@ struct BwdCfg {
   uint32_t stage_bytes;  // 2 * rps * row_bytes: rps x rows, then rps dy rows
   uint32_t gamma_bytes;  // gamma (or ones) in shared memory, slot order
   uint32_t ring_off, bar_off, red_off;
+  uint32_t ostage_bytes;  // per-group dx staging buffer (rps rows); 0: dx stored directly
+  uint32_t out_off;       // offset of the staging buffers
 };
 
 struct BwdArgs {
@@ -123,6 +125,11 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C.bar_off) + (size_t)g * 2 * C.stages;
   uint64_t* empty = full + C.stages;
   float2* red = reinterpret_cast<float2*>(smem + C.red_off) + (size_t)g * 2 * kRedSlots;
+  // dx goes through the group's staging buffer and out with one bulk copy per
+  // row block (full, contiguous lines instead of each thread's 16-byte
+  // pieces), when the plan gives one.
+  const bool bulk_out = C.ostage_bytes != 0;
+  const uint32_t ostage = smem_u32(smem + C.out_off + (size_t)g * C.ostage_bytes);
 
   const int64_t gg = (int64_t)g * gridDim.x + blockIdx.x;
   const int64_t rb_end = gg < C.ngt ? C.n_row_blocks : 0;
@@ -181,6 +188,10 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
     const uint32_t sx = smem_u32(st + (size_t)rs * C.row_bytes);
     const uint32_t sd = smem_u32(st + (size_t)(C.rps + rs) * C.row_bytes);
 
+    // The staging buffer is free again once the previous row block's bulk
+    // copy has read it; the group learns it at the __syncwarp below, or at
+    // the row sum's named barrier for rows of several warps.
+    if (bulk_out && issuer) bulk_wait_read_all();
     // ---- x and dy into registers, the stage straight back to the issuer
     uint32_t xr[BPT][16], dr[BPT][16];
 #pragma unroll
@@ -265,10 +276,28 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
           const __nv_bfloat162 h = __floats2bfloat162_rn(r.x, r.y);
           o[i] = *reinterpret_cast<const uint32_t*>(&h);
         }
-        if (blk) stg128_stream(dxrow + ((j + rot) & 3) * 8, make_uint4(o[0], o[1], o[2], o[3]));
+        if (blk) {
+          if (bulk_out)
+            sts128(ostage + (uint32_t)(rs * C.D + k * kBlock + ((j + rot) & 3) * 8) * 2u,
+                   make_uint4(o[0], o[1], o[2], o[3]));
+          else
+            stg128_stream(dxrow + ((j + rot) & 3) * 8, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+      }
+    }
+    if (bulk_out) {
+      fence_proxy_async_smem();
+      if (TPR > 32) named_barrier_sync(bar_id, TPR);
+      else __syncwarp();
+      if (issuer) {
+        const int64_t r0 = rb * C.rps;
+        const int64_t nrows = C.T - r0 < (int64_t)C.rps ? C.T - r0 : (int64_t)C.rps;
+        bulk_copy_s2g(A.dx + r0 * (int64_t)C.D, ostage, (uint32_t)nrows * C.row_bytes);
+        bulk_commit();
       }
     }
   }
+  if (bulk_out && issuer) bulk_wait_all();
 
   // ---- this group's partial dgamma row (row slot rs)
   if (A.partial != nullptr && gg < C.ngt) {

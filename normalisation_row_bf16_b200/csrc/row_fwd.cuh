@@ -47,6 +47,12 @@ enum PMode { kP1 = 1, kP2 = 2, kP4 = 4, kPInf = 0, kPGeneral = 3 };
 // of its row needs ~120 registers (512 threads), 2 blocks ~96 (640), 1 block
 // fits in 80 (768).
 __host__ __device__ constexpr int fwd_max_threads(int bpt) { return bpt >= 4 ? 512 : (bpt == 2 ? 640 : 768); }
+// Threads per CTA a kernel is compiled for (its __launch_bounds__).  One-warp
+// rows of 65..128 blocks of E4M3 codes with nearest-even rounding launch 384
+// threads, and are compiled for 384: up to 168 registers a thread.
+__host__ __device__ constexpr int fwd_launch_threads(int bpt, int tpr, bool sr, int elem) {
+  return (bpt >= 4 && tpr == 32 && !sr && elem == 0) ? 384 : fwd_max_threads(bpt);
+}
 constexpr int kRedSlots = 16;  // warps per row group, at most
 
 struct FwdCfg {
@@ -81,6 +87,7 @@ struct FwdArgs {
   float p, eps;
   int n_stat;             // statistic terms per row (K; D / 16 for NVFP4)
   double inv_n_stat;      // 1 / n_stat, correctly rounded (host)
+  float inv_k_pow2;       // 1 / n_stat when n_stat is a power of two, else 0
   int pmode;
   uint32_t seed_lo, seed_hi;
   int scale_mma;          // scales in the tcgen05 128x4 layout
@@ -156,26 +163,73 @@ __device__ __forceinline__ int ref_exponent(uint32_t mb) { return max((int)(mb >
 // hi + lo.
 constexpr float kSplitMagic = 1536.0f;   // 1.5 * 2^10: rounds to multiples of 2^-13
 
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<const float2*>(&d);
+}
+
 template <int BPT>
 __device__ __forceinline__ float2 pmean_split_sum(const uint32_t (&mb)[BPT], float inv, int pmode) {
-  float hs = 0.0f, ls = 0.0f;
+  // r = m * inv is exact (a power-of-two scaling into [0, 2)); t = r^2 (p = 2)
+  // or r * 1 (p = 1), which each fma forms exactly before its one rounding.
+  // Two terms per packed f32x2 instruction; (hi, lo) sums kept per lane of
+  // the pair, whose two hi (two lo) sums add exactly at the end.
+  const float2 inv2 = make_float2(inv, inv), mg = make_float2(kSplitMagic, kSplitMagic);
+  float2 hs = make_float2(0.0f, 0.0f), ls = make_float2(0.0f, 0.0f);
 #pragma unroll
-  for (int b = 0; b < BPT; ++b) {
-    const float r = bf16bits_to_float(mb[b]) * inv;
-    const float t = pmode == kP1 ? r : r * r;
-    const float hi = __fsub_rn(__fadd_rn(t, kSplitMagic), kSplitMagic);
-    hs = __fadd_rn(hs, hi);
-    ls = __fadd_rn(ls, __fsub_rn(t, hi));
+  for (int b = 0; b < BPT; b += 2) {
+    const float m0 = bf16bits_to_float(mb[b]), m1 = b + 1 < BPT ? bf16bits_to_float(mb[b + 1]) : 0.0f;
+    const float2 r = mul2(make_float2(m0, m1), inv2);
+    const float2 f = pmode == kP1 ? make_float2(1.0f, 1.0f) : r;
+    const float2 hi = add2(fma2(r, f, mg), make_float2(-kSplitMagic, -kSplitMagic));
+    hs = add2(hs, hi);
+    ls = add2(ls, fma2(r, f, make_float2(-hi.x, -hi.y)));
   }
-  return make_float2(hs, ls);
+  return make_float2(__fadd_rn(hs.x, hs.y), __fadd_rn(ls.x, ls.y));
+}
+
+// sqrt(q) rounded to fp32 for q = s + e held exactly as an fp32 pair with
+// |e| <= ulp(s) / 2, s in [2^-10, 4): g = the correctly rounded sqrt of s is
+// at most one step from the answer, and which step follows from the exact
+// residual s - g^2 (one fma: the residual of a correctly rounded square root
+// is representable) plus e, against g * ulp(g) (half for the step below a
+// power of two): sqrt(q) passes the midpoint g + ulp/2 iff q - g^2 exceeds
+// g * ulp + ulp^2 / 4.  The fp32 sum of residual and e errs by ~2^-23 of
+// g * ulp, so a decision within 2^-18 of a midpoint is left undecided
+// (returns false) for the caller's double-precision path.
+__device__ __forceinline__ bool sqrt_pair_rn(float s, float e, float& out) {
+  const float g = __fsqrt_rn(s);
+  const float d = __fadd_rn(__fmaf_rn(-g, g, s), e);        // q - g^2, rounded
+  const uint32_t gb = __float_as_uint(g);
+  const float u = __uint_as_float((gb & 0x7F800000u) - (23u << 23));   // ulp(g), g >= 2^-5
+  const float t_up = __fmul_rn(g, u);                        // g * ulp, exact
+  const bool pow2 = (gb & 0x7FFFFFu) == 0;
+  const float t_dn = pow2 ? 0.5f * t_up : t_up;              // g * (ulp below g)
+  const float band = t_up * 3.814697265625e-06f;            // 2^-18 * g * ulp
+  const bool near = fabsf(d - t_up) <= band || fabsf(d + t_dn) <= band;
+  out = d > t_up ? __fadd_rn(g, u) : (d < -t_dn ? __fsub_rn(g, pow2 ? 0.5f * u : u) : g);
+  return !near;
 }
 
 __device__ __forceinline__ float2 seg_sum2(float2 v, int width) {
-  for (int off = width >> 1; off > 0; off >>= 1) {
-    v.x = __fadd_rn(v.x, __shfl_xor_sync(0xFFFFFFFFu, v.x, off));
-    v.y = __fadd_rn(v.y, __shfl_xor_sync(0xFFFFFFFFu, v.y, off));
-  }
+  for (int off = width >> 1; off > 0; off >>= 1)
+    v = add2(v, make_float2(__shfl_xor_sync(0xFFFFFFFFu, v.x, off), __shfl_xor_sync(0xFFFFFFFFu, v.y, off)));
   return v;
+}
+
+// The p-mean's root in double from an exact (or double) sum S relative to
+// 2^(p E): the correctly rounded S / K, a correctly rounded square root (two
+// for p = 4), scaled and rounded once to fp32.  Kept out of line: rows of one
+// warp reach it only for shapes and values the fp32 path leaves to it.
+static __device__ __noinline__ float pmean_root_f64(double S, int pmode, int n_stat, double inv_n_stat, int E) {
+  const double Kd = (double)n_stat;
+  double q = S * inv_n_stat;
+  q = fma(fma(-q, Kd, S), inv_n_stat, q);   // the correctly rounded S / K
+  const double root = pmode == kP1 ? q : (pmode == kP2 ? sqrt(q) : sqrt(sqrt(q)));
+  return __double2float_rn(root * exp2_int_f64(E));
 }
 
 // G from this thread's block maxima (bf16 magnitude bits).
@@ -251,13 +305,34 @@ __device__ __forceinline__ float row_pmean(const uint32_t (&mb)[BPT], const FwdA
       else if (A.pmode != kPInf) Sf += red[w].y * exp2f(A.p * (float)d);
     }
   }
-  if (Mb >= 0x7F80u || A.pmode == kPInf) return bf16bits_to_float(Mb);  // inf / NaN / p = inf
+  const bool special = Mb >= 0x7F80u;       // inf / NaN: G is the maximum
+  if (split_p) {
+    // K a power of two: the sum as an fp32 pair sum + err, scaled by 1/K
+    // exactly; p = 1 takes its rounded value, p = 2 the pair's square root
+    // (sqrt_pair_rn); the result times 2^Ef is exact while it stays a normal
+    // fp32 number.  A row of one warp forms the pair by Fast2Sum of its hi and
+    // lo sums (hs >= 1, the warp maximum's own term, > |ls|: exact); a longer
+    // row splits its double sum (the pair then carries it to ~2^-48, far
+    // inside the band the root leaves undecided).  Anything else, and the rare
+    // undecided root, take the double path below (each warp decides alike).
+    float sum, err;
+    if (TPR > 32) {
+      sum = __double2float_rn(S);
+      err = __double2float_rn(S - (double)sum);
+    } else {
+      sum = __fadd_rn(s2.x, s2.y);
+      err = __fsub_rn(s2.y, __fsub_rn(sum, s2.x));
+    }
+    const float invK = A.inv_k_pow2;                          // 0 when K is not a power of two
+    float gu = __fmul_rn(sum, invK);
+    bool ok = invK != 0.0f && Ef >= -100;
+    if (A.pmode == kP2) ok = sqrt_pair_rn(gu, __fmul_rn(err, invK), gu) && ok;
+    if (__all_sync(0xFFFFFFFFu, ok || special))
+      return special ? bf16bits_to_float(Mb) : __fmul_rn(gu, exp2_int(Ef));
+  }
+  if (special || A.pmode == kPInf) return bf16bits_to_float(Mb);  // inf / NaN / p = inf
   if (!split_p && A.pmode != kP4) return powf(Sf / (float)A.n_stat, 1.0f / A.p) * exp2_int(Ef);
-  const double Kd = (double)A.n_stat, invK = A.inv_n_stat;
-  double q = S * invK;
-  q = fma(fma(-q, Kd, S), invK, q);      // the correctly rounded S / K
-  const double root = A.pmode == kP1 ? q : (A.pmode == kP2 ? sqrt(q) : sqrt(sqrt(q)));
-  return __double2float_rn(root * exp2_int_f64(Ef));
+  return pmean_root_f64(S, A.pmode, A.n_stat, A.inv_n_stat, Ef);
 }
 
 template <int TPR>
@@ -356,8 +431,12 @@ __device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a,
     }
   }
   if constexpr (ELEM == kElemE4M3) {
+    // a block holding NaN or infinity is rare: one vote instead of a select
+    // per word (every lane of the warp runs this together)
+    if (__any_sync(0xFFFFFFFFu, nan_block)) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) qw[i] = nan_block ? 0x7F7F7F7Fu : qw[i];
+      for (int i = 0; i < 8; ++i) qw[i] = nan_block ? 0x7F7F7F7Fu : qw[i];
+    }
   }
   return nan_block ? (uint8_t)0xFF : (uint8_t)(e + 127);
 }
@@ -503,8 +582,8 @@ __device__ __forceinline__ void gamma_slot(const uint8_t* smem, int K, int j, in
   }
 }
 
-template <int MODE, int TPR>
-constexpr bool kFwdBulkStores = (MODE != kModeRMSNorm) && (TPR > 32);
+template <int MODE, int TPR, bool SR>
+constexpr bool kFwdBulkStores = (MODE != kModeRMSNorm) && (TPR > 32) && !SR;
 
 // gamma sits in shared memory as fp32 for rows of up to 8192 elements (up to
 // 64 threads per row), as bf16 beyond.
@@ -514,7 +593,7 @@ __host__ __device__ constexpr bool gamma_fp32(int tpr) { return tpr == 0 || tpr 
 // for rows of fewer than 32 blocks, where C.tpr (< 32) rows share a warp.
 // HG: gamma given (MXNorm, RMSNorm); its shared-memory format follows TPR.
 template <int MODE, int BPT, int TPR, bool SR, bool HG, int ELEM>
-__global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const FwdArgs A, const FwdCfg C) {
+__global__ void __launch_bounds__(fwd_launch_threads(BPT, TPR, SR, ELEM), 1) row_fwd_kernel(const FwdArgs A, const FwdCfg C) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tpr = TPR ? TPR : C.tpr;
   const int gthreads = TPR ? TPR : 32;
@@ -535,9 +614,10 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
   // Rows of several warps (TPR > 32) stage their codes in the group's buffer
   // and write each row block with one bulk copy: full, contiguous lines for L2
   // and DRAM instead of each thread's 8-byte pieces (measured on B200 at
-  // 16384 x 16384: 154 -> 137 us; rows of one warp or less measured slightly
-  // faster with direct stores).  The plan gives the buffer when it fits.
-  const bool bulk_out = kFwdBulkStores<MODE, TPR> && C.ostage_bytes != 0;
+  // 16384 x 16384: 154 -> 137 us; rows of one warp or less, and stochastic
+  // rounding, whose arithmetic the extra barrier stalls, measured faster with
+  // direct stores).  The plan gives the buffer when it fits.
+  const bool bulk_out = kFwdBulkStores<MODE, TPR, SR> && C.ostage_bytes != 0;
   const uint32_t ostage = smem_u32(smem + C.out_off + (size_t)g * C.ostage_bytes);
   constexpr bool has_gamma = HG;   // MXNorm's gain, RMSNorm's, or a cast's (folded weight)
   constexpr bool kGF32 = gamma_fp32(TPR);
@@ -607,6 +687,10 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
     if (ok) ok = mbar_wait_bounded(&full[s], ph, A.status);
     const int64_t row = rb * C.rps + rs;
     const bool valid = row < C.T;
+    // scale byte offset of block k: row part once per row, then a few ops per
+    // block (row-major: row * K + k; tcgen05 layout: mma_scale_offset split
+    // into its row and k terms)
+    const int64_t srow_off = A.scale_mma ? mma_scale_offset(row, 0, A.kp4) : row * (int64_t)C.K;
     const uint32_t srow = smem_u32(ring + (size_t)s * C.stage_bytes + (size_t)rs * C.row_bytes);
 
     // ---- the row into registers, then the stage goes straight back to the
@@ -813,8 +897,7 @@ __global__ void __launch_bounds__(fwd_max_threads(BPT), 1) row_fwd_kernel(const 
               else
                 store_codes(A.q + row * (int64_t)C.D + (int64_t)k * kBlock, qw, rot);
             }
-            const int64_t so = A.scale_mma ? mma_scale_offset(row, k, A.kp4) : row * (int64_t)C.K + k;
-            A.scales[so] = code;
+            A.scales[srow_off + (A.scale_mma ? (int64_t)((k >> 2) * 512 + (k & 3)) : (int64_t)k)] = code;
           }
         }
       }
