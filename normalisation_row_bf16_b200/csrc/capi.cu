@@ -788,6 +788,13 @@ int mxnorm_set_tuning(int consumer_threads, int stages, int ctas_per_sm) {
   return MXN_OK;
 }
 
+int mxnorm_set_gemm_tiles(int mode) {
+  t_err.clear();
+  if (mode != 0 && mode != 1) return fail(MXN_ERR_ARG, "gemm tile mode = %d", mode);
+  gemm_mxfp8_set_pairs(mode);
+  return MXN_OK;
+}
+
 void mxnorm_debug_fail_next(int count) { t_fail_next = count > 0 ? count : 0; }
 
 }  // extern "C"

@@ -36,6 +36,15 @@
 #include "gemm_mxfp8.h"
 
 namespace mxn {
+
+// Process-wide switch of the tile shape (mxnorm_set_gemm_tiles).  Single-CTA
+// tiles by default: the pair kernel moves a third fewer operand bytes from L2
+// but measured slower on B200 (8192 x 6144 x 4096: 193 against 177 us under
+// ncu, tensor pipe active 52% against 57%).
+static int g_gemm_pairs = 0;
+void gemm_mxfp8_set_pairs(int on) { g_gemm_pairs = on ? 1 : 0; }
+static bool gemm_pair_enabled() { return g_gemm_pairs != 0; }
+
 namespace {
 
 constexpr int kTileM = 128, kTileN = 256, kTileK = 128;  // K elements (= bytes) per stage
@@ -332,6 +341,329 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 
+// ------------------------------------------------------------------ 2-SM tiles
+//
+// The same product on CTA pairs (a cluster of two CTAs on two SMs): each pair
+// owns a 256 x 256 output tile.  CTA r of the pair loads A rows 128 r .. of the
+// tile and B rows (output columns) 128 r .. of the tile into its own shared
+// memory, with their scale atoms; one thread of CTA 0 issues
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32), which reads A and B
+// from both CTAs' shared memory at the same offsets and accumulates rows
+// 128 r .. 128 r + 127 of the tile, all 256 columns, in CTA r's tensor memory.
+// Per output element the pair moves half the B operand a single-CTA 128 x 256
+// tile does: the L2 -> SM operand stream falls from (128 + 256) / (128 * 256)
+// to (256 + 256) / (256 * 256) bytes per output per K step, a third less.
+// Scales: CTA r holds the atom of its 128 A rows, and both B atoms of the tile
+// (all 256 columns: each CTA's accumulator spans every column), measured on
+// B200 -- with only its own B atom the other 128 columns came out wrong.
+//  * Both CTAs' tensor copies complete on CTA 0's "full" barrier (.cta_group::2
+//    copies; the barrier address is CTA 0's, found with mapa), which expects
+//    both halves' bytes.
+//  * CTA 0's MMA thread copies each CTA's scale atoms into that CTA's tensor
+//    memory (tcgen05.cp.cta_group::2), issues the MMAs and frees the stage in
+//    both CTAs with one tcgen05.commit per CTA (no multicast).
+//  * The epilogue warps of both CTAs read their own accumulator half and
+//    arrive on CTA 0's "accumulator empty" barrier (remote arrive from CTA 1).
+// Tensor memory is allocated and freed as a pair (tcgen05.alloc/dealloc
+// .cta_group::2 by warp 0 of both CTAs); a cluster barrier after set-up and
+// another before the free order everything that crosses the pair.  Every
+// mbarrier wait is bounded as in the single-CTA kernel.
+
+constexpr int kStages2 = 6;
+constexpr uint32_t kHalfBytes = 128 * kTileK;                // 16 KiB: 128 rows of A or of B
+constexpr uint32_t kAtomBytes = 512;                         // one 128 x 4 scale atom
+constexpr uint32_t kStageTx2 = 2u * (2u * kHalfBytes + 3u * kAtomBytes);   // both CTAs' bytes
+constexpr uint32_t kSfCol2 = 256;                            // scales: 12 columns per stage
+
+struct Smem2 {
+  uint8_t a[kStages2][kHalfBytes];                           // 1024-aligned (128B swizzle atoms)
+  uint8_t b[kStages2][kHalfBytes];
+  uint8_t sfa[kStages2][kAtomBytes];                         // this CTA's 128 A rows
+  uint8_t sfb[kStages2][2 * kAtomBytes];                     // all 256 B rows of the tile
+  uint64_t full[kStages2];                                   // CTA 0's: both halves' bytes
+  uint64_t empty[kStages2];                                  // each CTA's own
+  uint64_t acc_full;                                         // each CTA's own
+  uint64_t acc_empty;                                        // CTA 0's: both CTAs' epilogue warps
+  uint64_t mma_done;                                         // CTA 0's
+  uint32_t tmem_base;
+  uint32_t failed;
+  uint8_t cstage[kEpiWarps][32 * 64];
+};
+
+__device__ __forceinline__ bool failed_flag2(const Smem2& S) {
+  return *reinterpret_cast<const volatile uint32_t*>(&S.failed) != 0;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t n_clusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// Shared::cluster address of this CTA's shared-memory location `p` in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 2-D tensor copy into this CTA's shared memory, completing on the mbarrier at
+// shared::cluster address `bar` (CTA 0's).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t tmem, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(tmem), "l"(src_desc) : "memory");
+}
+
+// Arrive on the mbarrier at shared::cluster address `bar` once every prior
+// tcgen05 operation of this thread has completed.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Instruction descriptor of the pair MMA: M = 256, N = 256, otherwise as instr_desc.
+__device__ __forceinline__ uint32_t instr_desc_pair(uint32_t sf_id) {
+  return (sf_id << 4) | ((uint32_t)(256 >> 3) << 17) | (1u << 23) | ((uint32_t)(256 >> 4) << 24) | (sf_id << 29);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_mxfp8_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                           const __grid_constant__ CUtensorMap map_sa, const __grid_constant__ CUtensorMap map_sb,
+                           uint16_t* __restrict__ c, int M, int N, int K, unsigned* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // A launch without a two-CTA cluster would make the paired allocation below
+  // wait for a partner that does not exist: refuse it before anything else.
+  if (cluster_size() != 2) {
+    if (threadIdx.x == 0) atomicOr(status, kStatusWaitTimeout);
+    return;
+  }
+  Smem2& S = *reinterpret_cast<Smem2*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int m_tiles = M / 256;
+  const int n_tiles_all = m_tiles * (N / 256);
+  const int n_k = K / kTileK;
+  const int kp4 = K / 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    mbar_init(&S.acc_full, 1);
+    mbar_init(&S.acc_empty, 2 * kEpiWarps);
+    mbar_init(&S.mma_done, 1);
+    S.failed = 0;
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();                           // both CTAs' barriers and allocation are in place
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  griddep_wait();
+  griddep_launch_dependents();
+
+  const uint32_t cid = cluster_id_x(), ncl = n_clusters_x();
+  uint32_t n_issued = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      // ----------------------------------------------------- producer (both CTAs)
+      uint32_t g = 0;
+      bool ok = true;
+      for (int t = (int)cid; t < n_tiles_all && ok; t += (int)ncl) {
+        const int mt = t % m_tiles, nt = t / m_tiles;
+        const int arow = mt * 256 + (int)rank * 128, brow = nt * 256 + (int)rank * 128;
+        const int atile = 2 * mt + (int)rank;                                  // 128-row scale tiles
+        for (int kb = 0; kb < n_k; ++kb, ++g) {
+          const int s = (int)(g % kStages2);
+          const uint32_t ph = (g / kStages2) & 1u;
+          if (!mbar_wait_bounded(&S.empty[s], ph ^ 1u, status) || failed_flag2(S)) {
+            atomicOr(&S.failed, 1u);
+            ok = false;
+            break;
+          }
+          const uint32_t bar0 = cluster_addr(&S.full[s], 0);
+          if (rank == 0) mbar_arrive_expect_tx(&S.full[s], kStageTx2);
+          tma_load_2d_pair(S.a[s], &map_a, kb * kTileK, arow, bar0);
+          tma_load_2d_pair(S.b[s], &map_b, kb * kTileK, brow, bar0);
+          // scale atoms: atom (tile, kb) is rows 4 * (tile * kp4 / 4 + kb) .. + 3 of the 128-byte-row view
+          tma_load_2d_pair(S.sfa[s], &map_sa, 0, 4 * (atile * (kp4 / 4) + kb), bar0);
+          tma_load_2d_pair(S.sfb[s], &map_sb, 0, 4 * ((2 * nt) * (kp4 / 4) + kb), bar0);
+          tma_load_2d_pair(S.sfb[s] + kAtomBytes, &map_sb, 0, 4 * ((2 * nt + 1) * (kp4 / 4) + kb), bar0);
+          n_issued = g + 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------------- MMA (CTA 0)
+      const uint32_t empty1_base = cluster_addr(&S.empty[0], 1);
+      const uint32_t acc_full1 = cluster_addr(&S.acc_full, 1);
+      uint32_t g = 0, it = 0;
+      bool ok = true;
+      for (int t = (int)cid; t < n_tiles_all && ok; t += (int)ncl, ++it) {
+        if (!mbar_wait_bounded(&S.acc_empty, (it & 1u) ^ 1u, status) || failed_flag2(S)) {
+          atomicOr(&S.failed, 1u);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < n_k; ++kb, ++g) {
+          const int s = (int)(g % kStages2);
+          const uint32_t ph = (g / kStages2) & 1u;
+          if (!mbar_wait_bounded(&S.full[s], ph, status) || failed_flag2(S)) {
+            atomicOr(&S.failed, 1u);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa_col = kSfCol2 + (uint32_t)s * 12u, sfb_col = sfa_col + 4u;
+          tmem_cp_sf_pair(tmem + sfa_col, smem_desc(smem_u32(S.sfa[s]), 0, 128, 0));
+          tmem_cp_sf_pair(tmem + sfb_col, smem_desc(smem_u32(S.sfb[s]), 0, 128, 0));
+          tmem_cp_sf_pair(tmem + sfb_col + 4u, smem_desc(smem_u32(S.sfb[s] + kAtomBytes), 0, 128, 0));
+          const uint32_t a0 = smem_u32(S.a[s]), b0 = smem_u32(S.b[s]);
+#pragma unroll
+          for (int k = 0; k < kTileK / 32; ++k) {
+            const uint64_t ad = smem_desc(a0 + 32u * k, 16, 1024, 2);
+            const uint64_t bd = smem_desc(b0 + 32u * k, 16, 1024, 2);
+            mma_mxf8_pair(tmem + kAccCol, ad, bd, instr_desc_pair((uint32_t)k),
+                          (tmem + sfa_col) | ((uint32_t)k << 30), (tmem + sfb_col) | ((uint32_t)k << 30),
+                          (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          // the stage is free in both CTAs once these MMAs retire
+          tc_commit_pair(smem_u32(&S.empty[s]));
+          tc_commit_pair(empty1_base + (uint32_t)s * 8u);
+        }
+        if (ok) {
+          tc_commit_pair(smem_u32(&S.acc_full));
+          tc_commit_pair(acc_full1);
+        }
+      }
+      tc_commit_pair(smem_u32(&S.mma_done));
+      if (!ok) {                                 // wake both epilogues; they see the failure or time out
+        tc_commit_pair(smem_u32(&S.acc_full));
+        tc_commit_pair(acc_full1);
+      }
+    }
+  } else {
+    // ------------------------------------------------------ epilogue (both CTAs)
+    const int e = warp - 2;
+    const int quarter = warp & 3;
+    const int half = e >> 2;
+    const uint32_t acc_empty0 = cluster_addr(&S.acc_empty, 0);
+    uint32_t it = 0;
+    for (int t = (int)cid; t < n_tiles_all; t += (int)ncl, ++it) {
+      const int mt = t % m_tiles, nt = t / m_tiles;
+      const bool got = mbar_wait_bounded(&S.acc_full, it & 1u, status);
+      tc_fence_after();
+      if (!got || failed_flag2(S)) {
+        if (lane == 0) atomicOr(&S.failed, 1u);
+        break;
+      }
+      uint32_t r[4][32];
+      const uint32_t ta = tmem + kAccCol + (uint32_t)(half * 128) + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tmem_ld32(ta + 32u * j, r[j]);
+      tmem_ld_fence(r[0], true);
+#pragma unroll
+      for (int j = 1; j < 4; ++j) tmem_ld_fence(r[j], false);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {                           // CTA 0's MMA thread may overwrite the accumulators
+        if (rank == 0) mbar_arrive(&S.acc_empty);
+        else mbar_arrive_remote(acc_empty0);
+      }
+      uint8_t* stg = S.cstage[e];
+      const uint32_t stg_u32 = smem_u32(stg);
+      uint16_t* ctile = c + (size_t)(mt * 256 + (int)rank * 128 + quarter * 32) * N + (size_t)nt * 256 + half * 128;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t o[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[j][2 * i]), __uint_as_float(r[j][2 * i + 1]));
+          o[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t off = (uint32_t)lane * 64u + (uint32_t)((v ^ ((lane >> 1) & 3)) * 16);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg_u32 + off), "r"(o[4 * v]),
+                       "r"(o[4 * v + 1]), "r"(o[4 * v + 2]), "r"(o[4 * v + 3])
+                       : "memory");
+        }
+        __syncwarp();
+#pragma unroll
+        for (int t2 = 0; t2 < 4; ++t2) {
+          const int rr = t2 * 8 + (lane >> 2), cc = lane & 3;
+          const uint4 v4 = lds128(stg_u32 + (uint32_t)rr * 64u + (uint32_t)((cc ^ ((rr >> 1) & 3)) * 16));
+          *reinterpret_cast<uint4*>(ctile + (size_t)rr * N + 32 * j + 8 * cc) = v4;
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (rank == 0 && warp == 1 && lane == 0) mbar_wait_bounded(&S.mma_done, 0, status);
+  // After a failure CTA 0 waits (bounded) for the last phase of every stage
+  // its producer filled: both CTAs' copies of a stage complete there.
+  if (rank == 0 && warp == 0 && lane == 0 && failed_flag2(S))
+    for (uint32_t j = (n_issued > (uint32_t)kStages2 ? n_issued - kStages2 : 0); j < n_issued; ++j)
+      mbar_wait_bounded(&S.full[j % kStages2], (j / kStages2) & 1u, status);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();                           // no MMA, copy or remote arrive into either CTA remains
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -357,6 +689,81 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_ro
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over a scale array in the tcgen05 layout viewed as rows of 128
+// bytes: one 512-byte atom is a box of 4 rows (no swizzle).
+bool make_sf_map(CUtensorMap* map, const void* base, size_t bytes) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {128, (cuuint64_t)(bytes / 128)};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {128, 4};
+  const cuuint32_t elem[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Clusters of two CTAs of the pair kernel that fit on the device at once
+// (0 if none), looked up once per device.
+int pair_clusters(int dev) {
+  static int cached[64];
+  static bool have[64];
+  if (dev < 0 || dev >= 64) return 0;
+  if (have[dev]) return cached[dev];
+  int n = 0;
+  const size_t smem = sizeof(Smem2);
+  if (cudaFuncSetAttribute(gemm_mxfp8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void*)gemm_mxfp8_pair_kernel, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  cached[dev] = n;
+  have[dev] = true;
+  return n;
+}
+
+int launch_pair(const void* a_q, const void* a_s, const void* b_q, const void* b_s, void* c, int M, int N, int K,
+                int clusters, unsigned* status, cudaStream_t stream, const char** why) {
+  CUtensorMap ma, mb, msa, msb;
+  if (!make_map(&ma, a_q, M, K, 128) || !make_map(&mb, b_q, N, K, 128) ||
+      !make_sf_map(&msa, a_s, (size_t)M * (K / 32)) || !make_sf_map(&msb, b_s, (size_t)N * (K / 32))) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return -1;
+  }
+  const int tiles = (M / 256) * (N / 256);
+  const int ncl = tiles < clusters ? tiles : clusters;
+  uint16_t* cp = static_cast<uint16_t*>(c);
+  void* argv[] = {&ma, &mb, &msa, &msb, &cp, &M, &N, &K, &status};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * ncl);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = sizeof(Smem2);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelExC(&cfg, (const void*)gemm_mxfp8_pair_kernel, argv);
+  if (e != cudaSuccess) { *why = cudaGetErrorString(e); return (int)e; }
+  return 0;
+}
+
 }  // namespace
 
 size_t gemm_mxfp8_smem_bytes() { return sizeof(Smem) + 1024; }
@@ -364,6 +771,15 @@ size_t gemm_mxfp8_smem_bytes() { return sizeof(Smem) + 1024; }
 // Launch: returns 0, or -1 (tensor map could not be encoded) / cuda error code.
 int gemm_mxfp8_launch(const void* a_q, const void* a_s, const void* b_q, const void* b_s, void* c, int M,
                       int N, int K, int sms, unsigned* status, cudaStream_t stream, const char** why) {
+  // 256 x 256 tiles on CTA pairs where the shape allows and the device has room.
+  if (M % 256 == 0 && N % 256 == 0 && gemm_pair_enabled()) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+      const int ncl = pair_clusters(dev);
+      const int cap = sms / 2;
+      if (ncl > 0) return launch_pair(a_q, a_s, b_q, b_s, c, M, N, K, ncl < cap ? ncl : cap, status, stream, why);
+    }
+  }
   CUtensorMap ma, mb;
   if (!make_map(&ma, a_q, M, K, kTileM) || !make_map(&mb, b_q, N, K, kTileN)) {
     *why = "cuTensorMapEncodeTiled failed";

@@ -42,6 +42,7 @@ SIGNATURES = {
     "mxnorm_last_error": (ctypes.c_char_p, []),
     "mxnorm_device_status": (_I32, [_P]),
     "mxnorm_set_tuning": (_I32, [_I32, _I32, _I32]),
+    "mxnorm_set_gemm_tiles": (_I32, [_I32]),
     "mxnorm_debug_fail_next": (None, [_I32]),
     "mxnorm_debug_wait_timeout": (_I32, [_U64, _P, _P]),
 }
@@ -300,6 +301,11 @@ def device_status(stream=None) -> int:
 
 def set_tuning(consumer_threads: int = 0, stages: int = 0, ctas_per_sm: int = 0):
     _check(lib().mxnorm_set_tuning(consumer_threads, stages, ctas_per_sm))
+
+
+def set_gemm_tiles(mode: int = 0):
+    """0: single-CTA 128 x 256 GEMM tiles (default); 1: CTA-pair 256 x 256 tiles where M % 256 == 0."""
+    _check(lib().mxnorm_set_gemm_tiles(int(mode)))
 
 
 def debug_fail_next(count: int):
