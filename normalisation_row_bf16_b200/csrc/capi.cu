@@ -312,11 +312,20 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int
   const int64_t max_ctas = (int64_t)sms * occ;
   const int64_t need_ctas = (C.n_row_blocks + ng - 1) / ng;
   const int64_t ctas = need_ctas < max_ctas ? need_ctas : max_ctas;
-  // Every active group gets R or R - 1 row blocks with R = ceil(blocks / groups):
-  // only as many groups as R rounds need take rows, so no round runs on a
-  // fraction of the groups while the rest idle.
-  const int64_t R = (C.n_row_blocks + ctas * ng - 1) / (ctas * ng);
-  C.ngt = R > 0 ? (C.n_row_blocks + R - 1) / R : 0;
+  // Nearest-even E4M3 codes (memory-bound): every active group gets R or R - 1
+  // row blocks with R = ceil(blocks / groups), only as many groups as R rounds
+  // need take rows, so no round runs on a fraction of the groups while the
+  // rest idle.  Stochastic rounding and the FP4 formats (bound by their
+  // arithmetic): row blocks dealt round-robin over every group, which spreads
+  // them evenly over the SMs (within one block per SM) -- measured on B200 at
+  // 8192 x 4096: SR 55.4 -> 53.1, MXFP4 18.3 -> 17.6, NVFP4 24.8 -> 23.9 us,
+  // while the E4M3 forward ran 18.8 -> 19.5 us that way.
+  if (sr || elem != kElemE4M3) {
+    C.ngt = ctas * ng;
+  } else {
+    const int64_t R = (C.n_row_blocks + ctas * ng - 1) / (ctas * ng);
+    C.ngt = R > 0 ? (C.n_row_blocks + R - 1) / R : 0;
+  }
   P->grid = (int)ctas;
   return MXN_OK;
 }
