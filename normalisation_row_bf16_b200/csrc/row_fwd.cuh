@@ -157,10 +157,11 @@ __device__ __forceinline__ int ref_exponent(uint32_t mb) { return max((int)(mb >
 // and lo = t - hi, |lo| <= 2^-(g+1), with g = 13.  A warp adds at most 256
 // terms: the hi parts are multiples of 2^-13 below 2^10 (23 bits), and the lo
 // parts (below 2^-6 in all) stay exact while every term keeps its bits above
-// 2^-29 -- for p = 2 while no block maximum is below 2^-8 of the warp maximum,
-// for p = 1 below 2^-22 (a smaller term is added with an error below 2^-30 of
-// the largest one).  Two fp32 shuffle sums then carry the exact total as
-// hi + lo.
+// 2^-29 -- for p = 2 while no nonzero block maximum is below 2^-7 of the warp
+// maximum's power of two, for p = 1 below 2^-22.  The split flags a term
+// outside that range (one unsigned compare on the bf16 bits); a warp holding
+// one sums its terms in double instead (exact in double), a rare path.  Two
+// fp32 shuffle sums then carry the exact total as hi + lo.
 constexpr float kSplitMagic = 1536.0f;   // 1.5 * 2^10: rounds to multiples of 2^-13
 
 __device__ __forceinline__ float2 add2(float2 a, float2 b) {
@@ -172,7 +173,8 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
 }
 
 template <int BPT>
-__device__ __forceinline__ float2 pmean_split_sum(const uint32_t (&mb)[BPT], float inv, int pmode) {
+__device__ __forceinline__ float2 pmean_split_sum(const uint32_t (&mb)[BPT], float inv, int pmode,
+                                                  uint32_t tiny1, bool& inexact) {
   // r = m * inv is exact (a power-of-two scaling into [0, 2)); t = r^2 (p = 2)
   // or r * 1 (p = 1), which each fma forms exactly before its one rounding.
   // Two terms per packed f32x2 instruction; (hi, lo) sums kept per lane of
@@ -188,6 +190,12 @@ __device__ __forceinline__ float2 pmean_split_sum(const uint32_t (&mb)[BPT], flo
     hs = add2(hs, hi);
     ls = add2(ls, fma2(r, f, make_float2(-hi.x, -hi.y)));
   }
+  // 0 < m < the range's lower bound, on the bits: (m - 1) < (bound - 1)
+  // unsigned; zero maxima wrap to the top and never count
+  uint32_t lowest = mb[0] - 1u;
+#pragma unroll
+  for (int b = 1; b < BPT; ++b) lowest = min(lowest, mb[b] - 1u);
+  inexact = lowest < tiny1;
   return make_float2(__fadd_rn(hs.x, hs.y), __fadd_rn(ls.x, ls.y));
 }
 
@@ -262,23 +270,34 @@ __device__ __forceinline__ float row_pmean(const uint32_t (&mb)[BPT], const FwdA
   float2 s2 = make_float2(0.0f, 0.0f);   // p = 1, 2: the warp's exact sum as hi + lo
   double sd = 0.0;                       // p = 4: the warp's double sum
   float sw = 0.0f;                       // other p: the warp's fp32 sum
+  bool dp_sum = false;                   // p = 1, 2: the warp summed in double instead
+  bool use_f64 = A.pmode == kP4;
   if (split_p) {
-    s2 = seg_sum2(pmean_split_sum<BPT>(mb, inv, A.pmode), W);
-  } else if (A.pmode == kP4) {
+    // bf16 bits of the lower bound of the exact range: 2^(Ew - 7) for p = 2,
+    // 2^(Ew - 22) for p = 1 (minus one, for the unsigned compare)
+    const int eb = Ew + 127 - (A.pmode == kP2 ? 7 : 22);
+    const uint32_t tiny1 = eb > 0 ? ((uint32_t)eb << 7) - 1u : 0u;
+    bool inexact;
+    s2 = seg_sum2(pmean_split_sum<BPT>(mb, inv, A.pmode, tiny1, inexact), W);
+    dp_sum = use_f64 = __any_sync(0xFFFFFFFFu, inexact);
+  }
+  if (use_f64) {
+    // p = 4, or p = 1, 2 with a term outside the fp32 pair's exact range:
+    // (m / 2^E)^p in double (exact: at most 32 significant bits)
 #pragma unroll
     for (int b = 0; b < BPT; ++b) {
       const double r = (double)(bf16bits_to_float(mb[b]) * inv), r2 = r * r;
-      sd += r2 * r2;
+      sd += A.pmode == kP1 ? r : (A.pmode == kP2 ? r2 : r2 * r2);
     }
     sd = seg_sum_f64(sd, W);
-  } else if (A.pmode != kPInf) {
+  } else if (!split_p && A.pmode != kPInf) {
 #pragma unroll
     for (int b = 0; b < BPT; ++b) sw += powf(bf16bits_to_float(mb[b]) * inv, A.p);
     sw = seg_sum(sw, W);
   }
   uint32_t Mb = mloc;
   int Ef = Ew;
-  double S = split_p ? (double)s2.x + (double)s2.y : sd;
+  double S = (split_p && !dp_sum) ? (double)s2.x + (double)s2.y : sd;
   float Sf = sw;
   if (TPR > 32) {
     // slots 0..7: the warps' maxima (bf16 bits) and fp32 sums; 8..15: their
@@ -306,7 +325,7 @@ __device__ __forceinline__ float row_pmean(const uint32_t (&mb)[BPT], const FwdA
     }
   }
   const bool special = Mb >= 0x7F80u;       // inf / NaN: G is the maximum
-  if (split_p) {
+  if (split_p && !(TPR <= 32 && dp_sum)) {
     // K a power of two: the sum as an fp32 pair sum + err, scaled by 1/K
     // exactly; p = 1 takes its rounded value, p = 2 the pair's square root
     // (sqrt_pair_rn); the result times 2^Ef is exact while it stays a normal

@@ -118,6 +118,27 @@ def test_mxnorm_fwd_special_rows():
         assert Gh[0] == 0 and Gh[1] == 3.0
 
 
+@pytest.mark.parametrize("D", [512, 1024, 3072, 8192])
+@pytest.mark.parametrize("p", [2.0, 1.0, 4.0])
+def test_mxnorm_fwd_wide_range_rows(D, p):
+    """Rows whose block maxima span up to 2^-40 of the row maximum: the p-mean's
+    terms then fall outside the range the fp32 hi/lo sum holds exactly, and the
+    kernel sums them in double; the strict clause (scales and codes equal to the
+    oracle's own result) must still hold."""
+    T = 48
+    x = synthetic.activations(T, D, "normal", seed=D + 1)
+    gen = torch.Generator().manual_seed(D)
+    k = torch.randint(0, 41, (T, D // 32), generator=gen).float()
+    k[:, 0] = 0.0                                          # one block at full size per row
+    x = (x.float().view(T, D // 32, 32) * torch.exp2(-k)[:, :, None]).view(T, D).to(torch.bfloat16)
+    xd = _dev(x)
+    gd = _dev(synthetic.gamma(D, seed=D))
+    q, s, G = ops.mxnorm_fwd(xd, gd, p)
+    torch.cuda.synchronize()
+    rep = check_mxnorm_fwd(xd, gd, p, 0, 0, q, s, G)
+    assert rep["strict_G_bit_mismatch_rows"] == 0, rep
+
+
 def test_mxnorm_fwd_nonfinite_blocks():
     """Out of contract but defined: NaN/inf mark their blocks (scale 0xFF, code 0x7F)."""
     D = 128
@@ -134,18 +155,29 @@ def test_mxnorm_fwd_nonfinite_blocks():
 
 
 def test_mxnorm_fwd_mma_scale_layout():
+    """Scales in the tcgen05 128 x 4 layout: every (row, block) byte equals the
+    oracle's own scale (the strict clause), codes and G equal the row-major
+    call's, which is checked against the oracle, and the layout's padding rows
+    and columns stay untouched."""
     T, D = 300, 4128          # ragged in both padded dimensions
     x = _dev(synthetic.activations(T, D, "normal", seed=9))
     g = _dev(synthetic.gamma(D, seed=9))
-    q0, s0, G0 = ops.mxnorm_fwd(x, g, 2.0)
-    q1, s1, G1 = ops.mxnorm_fwd(x, g, 2.0, scale_layout=ops.SCALES_MMA)
-    torch.cuda.synchronize()
-    assert torch.equal(q0, q1) and torch.equal(G0, G1)
     K = D // 32
     kp4 = (K + 3) // 4 * 4
+    s1 = torch.full((ops.scales_bytes(T, D, ops.SCALES_MMA),), 0xAB, dtype=torch.uint8, device="cuda")
+    q1, s1, G1 = ops.mxnorm_fwd(x, g, 2.0, scale_layout=ops.SCALES_MMA, scales=s1)
+    q0, s0, G0 = ops.mxnorm_fwd(x, g, 2.0)
+    torch.cuda.synchronize()
+    check_mxnorm_fwd(x, g, 2.0, 0, 0, q0, s0, G0)
+    assert torch.equal(q1, q0) and torch.equal(G1, G0)
+    _, s_ref, _ = oracle.mxnorm_fwd(x.cpu(), g.cpu(), 2.0)
     rows, ks = np.meshgrid(np.arange(T), np.arange(K), indexing="ij")
     off = mma_scale_offset(rows, ks, kp4)
-    assert np.array_equal(to_np_u8(s1)[off], to_np_u8(s0))
+    sh = to_np_u8(s1)
+    assert np.array_equal(sh[off], s_ref)
+    untouched = np.ones(sh.size, bool)
+    untouched[off.ravel()] = False
+    assert np.all(sh[untouched] == 0xAB)
 
 
 # ------------------------------------------------------------------- MXCast
