@@ -478,19 +478,20 @@ __device__ __forceinline__ void stage_codes(uint32_t sa, const uint32_t (&qw)[8]
   for (int j = 0; j < 4; ++j) sts64(sa + (uint32_t)(((j + rot) & 3) * 8), qw[2 * j], qw[2 * j + 1]);
 }
 
-// bf16 magnitude bits of the two 16-element halves of a block held in slot
-// order (slot j holds chunk (j + rot) & 3; chunks 0-1 form half 0).  NaN
-// magnitudes compare above infinity, so a NaN stays the maximum.
-__device__ __forceinline__ void half_absmax_bits(const uint32_t (&w)[16], int rot, uint32_t& h0, uint32_t& h1) {
-  uint32_t sm[4];
+// bf16 magnitude bits of the two 16-element halves of an NVFP4 block held in
+// slot order (rotation 0 or 2: slots 0-1 hold one half, slots 2-3 the other;
+// hA is the half in slots 0-1).  NaN magnitudes compare above infinity, so a
+// NaN stays the maximum.
+__device__ __forceinline__ void half_absmax_bits(const uint32_t (&w)[16], uint32_t& hA, uint32_t& hB) {
+  uint32_t a[2];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t a = bf16x2_maxabs(bf16x2_maxabs(w[4 * j], w[4 * j + 1]), bf16x2_maxabs(w[4 * j + 2], w[4 * j + 3]));
-    sm[j] = max(a & 0x7FFFu, (a >> 16) & 0x7FFFu);
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t x = bf16x2_maxabs(bf16x2_maxabs(bf16x2_maxabs(w[8 * h], w[8 * h + 1]), bf16x2_maxabs(w[8 * h + 2], w[8 * h + 3])),
+                                     bf16x2_maxabs(bf16x2_maxabs(w[8 * h + 4], w[8 * h + 5]), bf16x2_maxabs(w[8 * h + 6], w[8 * h + 7])));
+    a[h] = max(x & 0x7FFFu, (x >> 16) & 0x7FFFu);
   }
-  const uint32_t p01 = max(sm[0], sm[1]), p12 = max(sm[1], sm[2]), p23 = max(sm[2], sm[3]), p30 = max(sm[3], sm[0]);
-  h0 = rot == 0 ? p01 : (rot == 1 ? p30 : (rot == 2 ? p23 : p12));
-  h1 = rot == 0 ? p23 : (rot == 1 ? p12 : (rot == 2 ? p01 : p30));
+  hA = a[0];
+  hB = a[1];
 }
 
 // NVFP4 quantisation of one 32-element block (two 16-element NVFP4 blocks)
@@ -522,21 +523,26 @@ template <bool SR>
 __device__ __forceinline__ uint32_t quantise_nvfp4(const float (&y)[32], const float (&sm)[4], int rot,
                                                    uint64_t idx0, const PhiloxKeys& pk, const float* rtab,
                                                    uint32_t (&qw)[8]) {
-  const float p01 = max3_abs_nan(sm[0], sm[1], 0.0f), p12 = max3_abs_nan(sm[1], sm[2], 0.0f);
-  const float p23 = max3_abs_nan(sm[2], sm[3], 0.0f), p30 = max3_abs_nan(sm[3], sm[0], 0.0f);
-  const float ah0 = rot == 0 ? p01 : (rot == 1 ? p30 : (rot == 2 ? p23 : p12));
-  const float ah1 = rot == 0 ? p23 : (rot == 1 ? p12 : (rot == 2 ? p01 : p30));
-  const bool bad0 = !(ah0 <= 3.402823466e38f), bad1 = !(ah1 <= 3.402823466e38f);   // NaN or infinity
-  const float s0 = bad0 ? 0.0f : nvfp4_scale_value(ah0), s1 = bad1 ? 0.0f : nvfp4_scale_value(ah1);
-  const uint32_t c0 = bad0 ? 0x7Fu : e4m3_code_of(s0), c1 = bad1 ? 0x7Fu : e4m3_code_of(s1);
-  const float inv0 = rtab[c0], inv1 = rtab[c1];
+  // Slot space (rotation 0 or 2): half A in slots 0-1, half B in slots 2-3;
+  // half A is the block's first half when rot == 0, its second when rot == 2.
+  float ah[2];
+  ah[0] = max3_abs_nan(sm[0], sm[1], 0.0f);
+  ah[1] = max3_abs_nan(sm[2], sm[3], 0.0f);
+  uint32_t code[2], and_mask[2], or_mask[2];
+  float inv[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const bool bad = !(ah[h] <= 3.402823466e38f);                  // NaN or infinity
+    code[h] = bad ? 0x7Fu : e4m3_code_of(nvfp4_scale_value(ah[h]));
+    inv[h] = rtab[code[h]];                                        // 0 for codes 0 and 0x7F
+    // a bad half's codes are all 0x7; a zero scale's are 0 (not -0)
+    and_mask[h] = bad ? 0u : (code[h] == 0 ? 0u : 0xFFFFFFFFu);
+    or_mask[h] = bad ? 0x77777777u : 0u;
+  }
 #pragma unroll
   for (int sl = 0; sl < 4; ++sl) {
-    const bool h1 = (((sl + rot) & 3) >> 1) != 0;
-    const float inv = h1 ? inv1 : inv0;
-    const bool bad = h1 ? bad1 : bad0;
-    const bool zero = (h1 ? c1 : c0) == 0;
-    const float2 inv2 = make_float2(inv, inv);
+    const int h = sl >> 1;
+    const float2 inv2 = make_float2(inv[h], inv[h]);
     float v[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -551,16 +557,17 @@ __device__ __forceinline__ uint32_t quantise_nvfp4(const float (&y)[32], const f
                      make_uint4((uint32_t)(ctr + 1), (uint32_t)((ctr + 1) >> 32), 0u, 0u)};
       philox4x32_10_x2(rr[0], rr[1], pk);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        v[4 * h] = sr_e2m1_grid(v[4 * h], rr[h].x);
-        v[4 * h + 1] = sr_e2m1_grid(v[4 * h + 1], rr[h].y);
-        v[4 * h + 2] = sr_e2m1_grid(v[4 * h + 2], rr[h].z);
-        v[4 * h + 3] = sr_e2m1_grid(v[4 * h + 3], rr[h].w);
+      for (int hh = 0; hh < 2; ++hh) {
+        v[4 * hh] = sr_e2m1_grid(v[4 * hh], rr[hh].x);
+        v[4 * hh + 1] = sr_e2m1_grid(v[4 * hh + 1], rr[hh].y);
+        v[4 * hh + 2] = sr_e2m1_grid(v[4 * hh + 2], rr[hh].z);
+        v[4 * hh + 3] = sr_e2m1_grid(v[4 * hh + 3], rr[hh].w);
       }
     }
-    qw[sl] = bad ? 0x77777777u : (zero ? 0u : cvt_e2m1x8_rn(v));
+    qw[sl] = (cvt_e2m1x8_rn(v) & and_mask[h]) | or_mask[h];
   }
-  return c0 | (c1 << 8);
+  // scale bytes in the block's order: half 0 in bits 0..7
+  return rot == 0 ? (code[0] | (code[1] << 8)) : (code[1] | (code[0] << 8));
 }
 
 // E2M1 codes of a block (16 bytes): slot j's word goes to bytes
@@ -603,6 +610,18 @@ __device__ __forceinline__ void gamma_slot(const uint8_t* smem, int K, int j, in
 
 template <int MODE, int TPR, bool SR>
 constexpr bool kFwdBulkStores = (MODE != kModeRMSNorm) && (TPR > 32) && !SR;
+
+// The chunk rotation of a thread's 64-byte blocks (slot j holds chunk
+// (j + rot) & 3), from its thread index or, identically, a block index: all
+// four rotations (eight threads of a shared-memory phase on eight distinct
+// bank groups) for E4M3 and E2M1; for NVFP4 only 0 and 2, so slots 0-1 and
+// 2-3 always hold the two 16-element halves and the per-half scale work needs
+// no per-thread selects (at the price of two-way bank conflicts on the row
+// loads).
+template <int ELEM>
+__device__ __forceinline__ int slot_rot(int x) {
+  return ELEM == kElemNVFP4 ? ((x >> 1) & 1) << 1 : (x >> 1) & 3;
+}
 
 // gamma sits in shared memory as fp32 for rows of up to 8192 elements (up to
 // 64 threads per row), as bf16 beyond.
@@ -672,7 +691,7 @@ __global__ void __launch_bounds__(fwd_launch_threads(BPT, TPR, SR, ELEM), 1) row
   if constexpr (has_gamma) {
     for (int i = tid; i < C.K * 4; i += blockDim.x) {
       const int k = i >> 2, j = i & 3;
-      const int c = (j + (k >> 1)) & 3;
+      const int c = (j + slot_rot<ELEM>(k)) & 3;
       const uint4 v = ldg128_nc(A.gamma + (size_t)k * kBlock + c * 8);
       if constexpr (kGF32) {
         const float4 lo = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
@@ -698,7 +717,7 @@ __global__ void __launch_bounds__(fwd_launch_threads(BPT, TPR, SR, ELEM), 1) row
   bool ok = true;
   int par = 0;
   const int bar_id = 1 + g;
-  const int rot = (tg >> 1) & 3;           // the same for every block of the thread
+  const int rot = slot_rot<ELEM>(tg);      // the same for every block of the thread
   int64_t it = 0;
   for (int64_t rb = gg; rb < rb_end; rb += C.ngt, ++it, par ^= 1) {
     const int s = (int)(it % C.stages);
@@ -770,7 +789,7 @@ __global__ void __launch_bounds__(fwd_launch_threads(BPT, TPR, SR, ELEM), 1) row
           }
         }
       } else if constexpr (ELEM == kElemNVFP4) {
-        half_absmax_bits(xr[b], rot, mh[b][0], mh[b][1]);   // NVFP4 blocks are the halves
+        half_absmax_bits(xr[b], mh[b][0], mh[b][1]);        // NVFP4 blocks are the halves
         mb[b] = max(mh[b][0], mh[b][1]);
       } else {
         mb[b] = block_absmax16(xr[b]);
