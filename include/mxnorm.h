@@ -222,8 +222,9 @@ int rmsnorm_then_mxcast(const void* x, const void* gamma, float eps, void* y_tmp
  * dgamma  bf16 [D] (written) or NULL; must be NULL when gamma is NULL.
  *         Deterministic: partial sums in a fixed order, no atomics.
  * workspace  device scratch of at least mxnorm_bwd_workspace_size(T, D)
- *         bytes (fp32 partial sums), 16-byte aligned; may be NULL when dgamma
- *         is NULL.  Contents on entry are ignored.
+ *         bytes (fp32 partial sums, one row of D per CTA of the launch),
+ *         16-byte aligned; may be NULL when dgamma is NULL.  Contents on
+ *         entry are ignored.
  */
 int mxnorm_bwd(const void* x, const void* dy, const void* gamma, const float* G, void* dx,
                void* dgamma, int64_t T, int64_t D, void* workspace, size_t workspace_bytes,
@@ -267,9 +268,8 @@ int mxfp8_gemm(const void* a_q, const void* a_s, const void* b_q, const void* b_
  * stays until the process exits -- so every process that uses the library,
  * each rank of a multi-GPU job included, holds 8 MiB on each device it uses.
  * The call allocates nothing.  To fit the scratch it may launch fewer CTAs
- * than mxnorm_bwd (every active row group writes its partial rows of D fp32,
- * at most 2^21 / D rows in all); it returns MXN_ERR_UNSUPPORTED if even one
- * CTA's partial rows would not fit.
+ * than mxnorm_bwd (every CTA writes one partial row of D fp32, at most
+ * 2^21 / D rows in all, which is at least 128 at D <= 16384).
  * The first call on a device looks up the scratch array's device address
  * (cudaGetSymbolAddress); make that first call outside any stream capture.
  * Every call on a device shares the one scratch array: calls that may overlap

@@ -362,7 +362,7 @@ struct BwdPlan {
   int threads = 0;
   size_t smem = 0;
   int grid = 0;
-  size_t partial_rows() const { return (size_t)C.ngt * (size_t)C.rps; }
+  size_t partial_rows() const { return (size_t)grid; }   // one per CTA
 };
 
 // Rows of up to 256 blocks: one block per thread (tpr = K, several rows per
@@ -402,7 +402,7 @@ int plan_bwd(int64_t T, int D, int sms, BwdPlan* P, int64_t max_partial_rows = 0
   // the buffers fit beside the rings of the planned groups.
   C.ostage_bytes = (uint32_t)align_up((size_t)C.rps * C.row_bytes, 128);
   auto smem_of = [&](int n) {
-    return (size_t)C.gamma_bytes + (size_t)n * stages * (C.stage_bytes + 2 * sizeof(uint64_t)) +
+    return (size_t)C.gamma_bytes + (size_t)n * stages * (C.stage_bytes + 2 * sizeof(uint64_t) + sizeof(uint32_t)) +
            (size_t)n * (per_group_fixed + C.ostage_bytes) + 128 + 16;
   };
   {
@@ -421,7 +421,8 @@ int plan_bwd(int64_t T, int D, int sms, BwdPlan* P, int64_t max_partial_rows = 0
   C.out_off = (uint32_t)align_up(C.ring_off + (size_t)ng * stages * C.stage_bytes, 128);
   C.bar_off = (uint32_t)align_up(C.out_off + (size_t)ng * C.ostage_bytes, 16);
   C.red_off = C.bar_off + (uint32_t)(ng * 2 * stages * sizeof(uint64_t));
-  P->smem = C.red_off + (size_t)ng * 2 * kRedSlots * sizeof(float2);
+  C.cnt_off = C.red_off + (uint32_t)(ng * 2 * kRedSlots * sizeof(float2));
+  P->smem = C.cnt_off + (size_t)ng * stages * sizeof(uint32_t);
   P->threads = ng * C.gthreads;
   P->kernel = pick_bwd_shape(bpt, C.tpr);
   if (!P->kernel) return fail(MXN_ERR_UNSUPPORTED, "mxnorm_bwd: no kernel for D = %d", D);
@@ -432,13 +433,7 @@ int plan_bwd(int64_t T, int D, int sms, BwdPlan* P, int64_t max_partial_rows = 0
   if (g_tuning.ctas_per_sm && g_tuning.ctas_per_sm < occ) occ = g_tuning.ctas_per_sm;
   int64_t ctas = (C.n_row_blocks + ng - 1) / ng;
   if (ctas > (int64_t)sms * occ) ctas = (int64_t)sms * occ;
-  if (max_partial_rows > 0) {
-    const int64_t cap = max_partial_rows / ((int64_t)ng * C.rps);
-    if (cap < 1)
-      return fail(MXN_ERR_UNSUPPORTED, "%lld partial rows per CTA exceed the scratch",
-                  (long long)((int64_t)ng * C.rps));
-    if (ctas > cap) ctas = cap;
-  }
+  if (max_partial_rows > 0 && ctas > max_partial_rows) ctas = max_partial_rows;   // one partial row per CTA
   const int64_t R = (C.n_row_blocks + ctas * ng - 1) / (ctas * ng);
   C.ngt = R > 0 ? (C.n_row_blocks + R - 1) / R : 0;
   P->grid = (int)ctas;
@@ -705,9 +700,9 @@ int mxnorm_bwd_noalloc(const void* x, const void* dy, const void* gamma, const f
   if (T == 0) return MXN_OK;
   DeviceInfo dev;
   if ((rc = device_info(&dev))) return rc;
-  // Each active row group writes rps partial rows of D floats: plan no more
-  // of them than the scratch holds (the kernel is persistent, so fewer groups
-  // cover all rows).
+  // Each CTA writes one partial row of D floats: plan no more CTAs than the
+  // scratch holds rows (the kernel is persistent, so fewer CTAs cover all
+  // rows).
   BwdPlan P;
   if ((rc = plan_bwd(T, (int)D, dev.sms, &P, dgamma ? (int64_t)(kNoAllocScratchFloats / (size_t)D) : 0)))
     return rc;

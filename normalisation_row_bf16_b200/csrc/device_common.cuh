@@ -23,6 +23,19 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Shared-memory counter add with acquire-release semantics at CTA scope:
+// returns the old value.  The warp that brings a count to its total sees
+// every earlier adder's prior accesses (here, its shared-memory reads of a
+// stage) as complete.
+__device__ __forceinline__ uint32_t smem_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "r"(smem_u32(p)), "r"(v)
+               : "memory");
+  return old;
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -129,12 +142,11 @@ __device__ __forceinline__ void bulk_copy_s2g(void* gmem_dst, uint32_t smem_src,
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every committed shared -> global copy of this thread has read its
-// source (the buffer may be rewritten) ...
+// source: the buffer may then be rewritten, or the CTA exit (the writes
+// themselves complete with the grid, before any dependent grid runs).
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
-// ... or has completed its writes.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Order this thread's shared-memory writes before later bulk copies that read them.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

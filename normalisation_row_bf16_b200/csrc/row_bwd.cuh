@@ -18,12 +18,15 @@
 //    1-D bulk copies that the group's first thread issues, completing on the
 //    group's own mbarriers;
 //  * a thread copies its x and dy blocks into registers and hands the stage
-//    back at once; G is fetched before the row's wait; products run as packed
-//    fp32 pairs; the two row sums (x . x, x . g) reduce with shuffles, plus
-//    shared memory and a named barrier when a row spans several warps.
-// At the end every active group writes its partial dgamma row(s) to the
-// workspace and dgamma_reduce_kernel adds them in a fixed order
-// (deterministic, no atomics).
+//    back after the first pass over them (in a row of several warps, the last
+//    warp to get there issues the refill, so no warp waits for the others); G is fetched
+//    before the row's wait; products run as packed fp32 pairs; the two row
+//    sums (x . x, x . g) reduce with shuffles, plus shared memory and a named
+//    barrier when a row spans several warps.
+// At the end the CTA adds its groups' dgamma partial sums in shared memory
+// (group order, fixed) and writes one partial row to the workspace;
+// dgamma_reduce_kernel then adds the CTAs' rows in a fixed order
+// (deterministic, no atomics on the sums).
 #pragma once
 
 #include "row_fwd.cuh"
@@ -51,6 +54,7 @@ struct BwdCfg {
   uint32_t ring_off, bar_off, red_off;
   uint32_t ostage_bytes;  // per-group dx staging buffer (rps rows); 0: dx stored directly
   uint32_t out_off;       // offset of the staging buffers
+  uint32_t cnt_off;       // per group and stage: warps done with the stage (rows of several warps)
 };
 
 struct BwdArgs {
@@ -59,7 +63,7 @@ struct BwdArgs {
   const uint16_t* gamma;  // bf16 [D] or null
   const float* G;         // fp32 [T]
   uint16_t* dx;           // bf16 [T, D]
-  float* partial;         // fp32 [ngt * rps, D] or null (no dgamma)
+  float* partial;         // fp32 [gridDim.x, D] or null (no dgamma): one partial row per CTA
   unsigned* status;
 };
 
@@ -125,6 +129,7 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C.bar_off) + (size_t)g * 2 * C.stages;
   uint64_t* empty = full + C.stages;
   float2* red = reinterpret_cast<float2*>(smem + C.red_off) + (size_t)g * 2 * kRedSlots;
+  uint32_t* done = reinterpret_cast<uint32_t*>(smem + C.cnt_off) + (size_t)g * C.stages;
   // dx goes through the group's staging buffer and out with one bulk copy per
   // row block (full, contiguous lines instead of each thread's 16-byte
   // pieces), when the plan gives one.
@@ -138,6 +143,7 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
     for (int s = 0; s < C.stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], n_gwarps);
+      done[s] = 0u;
     }
     fence_barrier_init();
   }
@@ -192,7 +198,7 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
     // copy has read it; the group learns it at the __syncwarp below, or at
     // the row sum's named barrier for rows of several warps.
     if (bulk_out && issuer) bulk_wait_read_all();
-    // ---- x and dy into registers, the stage straight back to the issuer
+    // ---- x and dy into registers
     uint32_t xr[BPT][16], dr[BPT][16];
 #pragma unroll
     for (int b = 0; b < BPT; ++b) {
@@ -207,16 +213,7 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
         dr[b][4 * j] = d.x; dr[b][4 * j + 1] = d.y; dr[b][4 * j + 2] = d.z; dr[b][4 * j + 3] = d.w;
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-    // Refill: a one-warp row refills at once; a row of several warps after the
-    // row sum below, whose named barrier every warp reaches only after it has
-    // released the stage -- so the issuer's wait never holds up its warp.
     const int64_t nrb = rb + (int64_t)C.stages * C.ngt;
-    if (TPR <= 32 && issuer && nrb < C.n_row_blocks) {
-      if (ok) ok = mbar_wait_bounded(&empty[s], ph, A.status);
-      if (ok) issue_bwd_block(A, C, nrb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
-    }
 
     // ---- pass 1: x . x and x . g (g = gamma * dy), and the dgamma partials
     // dy * x / G (they need only G, which is known before the row arrives)
@@ -244,12 +241,28 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
         }
       }
     }
+    // Refill, once pass 1 has used every register read from the stage (so
+    // those shared-memory reads are complete) and behind a proxy fence that
+    // orders them before the bulk copy overwriting the stage.  A one-warp row
+    // refills at once; in a row of several warps each warp counts itself done,
+    // and the one that completes the count issues the refill (the
+    // acquire-release add orders every warp's reads before it).
+    fence_proxy_async_smem();
+    __syncwarp();
+    if constexpr (TPR > 32) {
+      if (lane == 0 && smem_add_acq_rel(&done[s], 1u) == (uint32_t)(n_gwarps - 1)) {
+        done[s] = 0u;   // next added to after this stage's next fill completes
+        if (ok && nrb < C.n_row_blocks) issue_bwd_block(A, C, nrb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
+      }
+    } else {
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (issuer && nrb < C.n_row_blocks) {
+        if (ok) ok = mbar_wait_bounded(&empty[s], ph, A.status);
+        if (ok) issue_bwd_block(A, C, nrb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
+      }
+    }
     const float2 tot = row_sum2<TPR>(make_float2(xx.x + xx.y, xg.x + xg.y), C, red + par * kRedSlots,
                                      bar_id, wig, lane);
-    if (TPR > 32 && issuer && nrb < C.n_row_blocks) {
-      if (ok) ok = mbar_wait_bounded(&empty[s], ph, A.status);
-      if (ok) issue_bwd_block(A, C, nrb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
-    }
 
     // ---- pass 2: dx (zero for a row with G = 0 or x = 0)
     const bool live = valid && (G != 0.0f) && (tot.x != 0.0f);
@@ -297,15 +310,38 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
       }
     }
   }
-  if (bulk_out && issuer) bulk_wait_all();
+  if (bulk_out && issuer) bulk_wait_read_all();   // staging buffers read before exit
+  // Leave no copy in flight: the issuer waits for the last phase of every stage
+  // filled (already complete unless a wait gave up above).
+  if (issuer && !ok) {
+    for (int s = 0; s < C.stages; ++s) {
+      const int64_t last_it = it - 1 - ((it - 1 - s) % C.stages + C.stages) % C.stages;
+      if (last_it >= 0) mbar_wait_bounded(&full[s], (uint32_t)((last_it / C.stages) & 1), A.status);
+    }
+  }
+  if (A.partial == nullptr) return;
 
-  // ---- this group's partial dgamma row (row slot rs)
-  if (A.partial != nullptr && gg < C.ngt) {
+  // ---- the CTA's partial dgamma row.  Rows sharing a warp first fold their
+  // row slots together (xor butterfly over the slot bits of the lane); each
+  // group then puts its sums into its own idle ring (D floats fit in one
+  // stage), and the CTA adds the groups in group order.
+  if (TPR == 0) {
+    for (int m = tpr; m < 32; m <<= 1) {
+#pragma unroll
+      for (int b = 0; b < BPT; ++b)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[b][i] += __shfl_xor_sync(0xFFFFFFFFu, acc[b][i], m);
+    }
+  }
+  __syncthreads();                          // every group is past its last row
+  float* gsum = reinterpret_cast<float*>(smem + C.ring_off);   // row g at g * stages * stage_bytes
+  const size_t gstride = (size_t)C.stages * C.stage_bytes / sizeof(float);
+  if (rs == 0) {
 #pragma unroll
     for (int b = 0; b < BPT; ++b) {
       const int k = tg + b * tpr;
       if (k < C.K) {
-        float* prow = A.partial + ((int64_t)gg * C.rps + rs) * C.D + (int64_t)k * kBlock;
+        float* prow = gsum + (size_t)g * gstride + (size_t)k * kBlock;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           float* p = prow + ((j + rot) & 3) * 8;
@@ -317,13 +353,15 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
       }
     }
   }
-  // Leave no copy in flight: the issuer waits for the last phase of every stage
-  // it filled (already complete unless a wait gave up above).
-  if (issuer && !ok) {
-    for (int s = 0; s < C.stages; ++s) {
-      const int64_t last_it = it - 1 - ((it - 1 - s) % C.stages + C.stages) % C.stages;
-      if (last_it >= 0) mbar_wait_bounded(&full[s], (uint32_t)((last_it / C.stages) & 1), A.status);
+  __syncthreads();
+  float4* out = reinterpret_cast<float4*>(A.partial + (int64_t)blockIdx.x * C.D);
+  for (int c = tid; c < C.D / 4; c += blockDim.x) {
+    float4 v = reinterpret_cast<const float4*>(gsum)[c];
+    for (int q = 1; q < C.ng; ++q) {
+      const float4 w = reinterpret_cast<const float4*>(gsum + (size_t)q * gstride)[c];
+      v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
     }
+    out[c] = v;
   }
 }
 

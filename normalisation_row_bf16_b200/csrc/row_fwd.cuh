@@ -20,9 +20,12 @@
 //    mbarriers: no group ever waits for another, and the bytes in flight do not
 //    depend on register occupancy.
 //  * A thread copies its blocks from the stage into registers and hands the
-//    stage straight back; the refill (row block rb + stages * ngt) is issued
-//    before the row's arithmetic, so each group keeps `stages` rows of compute
-//    as look-ahead whatever the occupancy.  A thread reads its 64-byte block
+//    stage back after the block maxima (which use every register it read:
+//    the reads are then complete) behind a proxy fence ordering its
+//    shared-memory reads before the refill's bulk copy; the refill (row block
+//    rb + stages * ngt) is issued before the rest of the row's arithmetic, so
+//    each group keeps `stages` rows of compute as look-ahead whatever the
+//    occupancy.  A thread reads its 64-byte block
 //    as four 16-byte chunks in the order (j + k/2) mod 4, which puts the eight
 //    threads of a shared-memory phase on eight distinct bank groups.
 //  * gamma is converted once per CTA into shared memory in "slot order": the
@@ -731,9 +734,9 @@ __global__ void __launch_bounds__(fwd_launch_threads(BPT, TPR, SR, ELEM), 1) row
     const int64_t srow_off = A.scale_mma ? mma_scale_offset(row, 0, A.kp4) : row * (int64_t)C.K;
     const uint32_t srow = smem_u32(ring + (size_t)s * C.stage_bytes + (size_t)rs * C.row_bytes);
 
-    // ---- the row into registers, then the stage goes straight back to the
-    // issuer, so the copy of row block rb + stages * ngt overlaps this row's
-    // arithmetic (look-ahead = `stages` rows of compute).
+    // ---- the row into registers; after the block maxima the stage goes back
+    // to the issuer, so the copy of row block rb + stages * ngt overlaps the
+    // rest of this row's arithmetic.
     // (RMSNorm keeps the row in the stage instead: it reads it twice and hands
     // the stage back after its second pass, which needs far fewer registers.)
     constexpr bool kHold = (MODE != kModeRMSNorm);
@@ -755,16 +758,6 @@ __global__ void __launch_bounds__(fwd_launch_threads(BPT, TPR, SR, ELEM), 1) row
           xr[b][4 * j] = v.x; xr[b][4 * j + 1] = v.y; xr[b][4 * j + 2] = v.z; xr[b][4 * j + 3] = v.w;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      if (issuer) {
-        const int64_t nrb = rb + (int64_t)C.stages * C.ngt;
-        if (nrb < C.n_row_blocks) {
-          if (ok) ok = mbar_wait_bounded(&empty[s], ph, A.status);
-          if (ok) issue_row_block(A.x, C, nrb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
-        }
-      }
-      if (TPR > 32 && bulk_out) named_barrier_sync(bar_id, TPR);
     }
 
     // ---- pass 1: block maxima (MXNorm, Cast) or sum of squares (RMSNorm)
@@ -794,6 +787,23 @@ __global__ void __launch_bounds__(fwd_launch_threads(BPT, TPR, SR, ELEM), 1) row
       } else {
         mb[b] = block_absmax16(xr[b]);
       }
+    }
+    if constexpr (kHold) {
+      // Hand the stage back once pass 1 has used every register read from it
+      // (so those shared-memory reads are complete), behind a proxy fence that
+      // orders them before the bulk copy that overwrites the stage: without
+      // both, a refill could land before a slow ld.shared had read its data.
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (issuer) {
+        const int64_t nrb = rb + (int64_t)C.stages * C.ngt;
+        if (nrb < C.n_row_blocks) {
+          if (ok) ok = mbar_wait_bounded(&empty[s], ph, A.status);
+          if (ok) issue_row_block(A.x, C, nrb, ring + (size_t)s * C.stage_bytes, &full[s], pol);
+        }
+      }
+      if (TPR > 32 && bulk_out) named_barrier_sync(bar_id, TPR);
     }
 
     float2* redp = red + par * kRedSlots;
@@ -825,6 +835,7 @@ __global__ void __launch_bounds__(fwd_launch_threads(BPT, TPR, SR, ELEM), 1) row
           if (blk) stg128_stream(yrow + ((j + rot) & 3) * 8, make_uint4(o[0], o[1], o[2], o[3]));
         }
       }
+      fence_proxy_async_smem();   // this thread's reads of the stage before its refill
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
       if (issuer) {
@@ -955,10 +966,10 @@ __global__ void __launch_bounds__(fwd_launch_threads(BPT, TPR, SR, ELEM), 1) row
     }
 
   }
-  // Leave no copy in flight: the issuer waits for its bulk stores to complete
-  // and for the last phase of every stage it filled (already complete unless a
-  // wait gave up above).
-  if (bulk_out && issuer) bulk_wait_all();
+  // Leave no copy in flight: the issuer waits for its bulk stores to have read
+  // the staging buffer and for the last phase of every stage it filled
+  // (already complete unless a wait gave up above).
+  if (bulk_out && issuer) bulk_wait_read_all();   // staging buffers read before exit
   if (issuer && !ok) {
     for (int s = 0; s < C.stages; ++s) {
       const int64_t last_it = it - 1 - ((it - 1 - s) % C.stages + C.stages) % C.stages;
