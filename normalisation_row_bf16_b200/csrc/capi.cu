@@ -397,7 +397,7 @@ int plan_bwd(int64_t T, int D, int sms, BwdPlan* P, int64_t max_partial_rows = 0
   // One stage per group measured best on B200 (8192 x 4096: 47.4 us against
   // 49.1 with two stages and 51.6 with three groups of two stages).
   const int stages = g_tuning.stages ? g_tuning.stages : 1;
-  C.gamma_bytes = (uint32_t)align_up(2u * (uint32_t)D, 128);
+  C.gamma_bytes = (uint32_t)align_up(4u * (uint32_t)D, 128);   // fp32
   // dx staged per group and written with one bulk copy per row block, while
   // the buffers fit beside the rings of the planned groups.
   C.ostage_bytes = (uint32_t)align_up((size_t)C.rps * C.row_bytes, 128);
@@ -467,7 +467,7 @@ int launch_bwd(const BwdPlan& P, const BwdArgs& A, uint16_t* dgamma, cudaStream_
 
 // ----------------------------------------------- allocation-free backward
 //
-// Scratch for mxnorm_bwd_noalloc: the per-row-group dgamma partial sums, 2^21 fp32
+// Scratch for mxnorm_bwd_noalloc: the per-CTA dgamma partial sums, 2^21 fp32
 // (8 MiB).  The runtime reserves it on a device when the library's kernels are
 // first used there (whether or not mxnorm_bwd_noalloc is called) and holds it
 // until the process exits.  In host code the name is only a host-side stand-in; its device

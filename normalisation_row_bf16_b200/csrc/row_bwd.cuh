@@ -50,7 +50,7 @@ struct BwdCfg {
   int stages;            // ring depth per group
   uint32_t row_bytes;    // 2 * D
   uint32_t stage_bytes;  // 2 * rps * row_bytes: rps x rows, then rps dy rows
-  uint32_t gamma_bytes;  // gamma (or ones) in shared memory, slot order
+  uint32_t gamma_bytes;  // gamma (or ones) as fp32 in shared memory, slot order
   uint32_t ring_off, bar_off, red_off;
   uint32_t ostage_bytes;  // per-group dx staging buffer (rps rows); 0: dx stored directly
   uint32_t out_off;       // offset of the staging buffers
@@ -156,17 +156,21 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
     }
   }
 
-  // gamma (ones when NULL) into shared memory once per CTA in slot order: the
-  // 16 bytes that match x chunk slot j of block k at (j * K + k) * 16, so a
-  // warp's reads of one slot fall on consecutive words (registers stay free
-  // for x, dy and the dgamma sums).
+  // gamma (ones when NULL) into shared memory once per CTA, as fp32 in slot
+  // order: the first and second halves of x chunk slot j of block k at
+  // ((2j + h) * K + k) * 16, so a warp's reads of one slot fall on
+  // consecutive words and no thread converts gamma per row (registers stay
+  // free for x, dy and the dgamma sums).
   const int rot = (tg >> 1) & 3;
   for (int i = tid; i < C.K * 4; i += blockDim.x) {
     const int k = i >> 2, j = i & 3;
     const int c = (j + (k >> 1)) & 3;
     uint4 v = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
     if (A.gamma != nullptr) v = ldg128_nc(A.gamma + (size_t)k * kBlock + c * 8);
-    *reinterpret_cast<uint4*>(smem + ((size_t)j * C.K + k) * 16) = v;
+    *reinterpret_cast<float4*>(smem + ((size_t)(2 * j) * C.K + k) * 16) =
+        make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
+    *reinterpret_cast<float4*>(smem + ((size_t)(2 * j + 1) * C.K + k) * 16) =
+        make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
   }
   float acc[BPT][32];
 #pragma unroll
@@ -216,7 +220,9 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
     const int64_t nrb = rb + (int64_t)C.stages * C.ngt;
 
     // ---- pass 1: x . x and x . g (g = gamma * dy), and the dgamma partials
-    // dy * x / G (they need only G, which is known before the row arrives)
+    // dy * x / G (they need only G, which is known before the row arrives).
+    // dy * x is exact in fp32 (two 8-bit significands), so x . g adds the
+    // same exact terms x * gamma * dy as a sum over x * (gamma * dy) would.
     const float invG = (G != 0.0f) ? __frcp_rn(G) : 0.0f;
     const float2 invG2 = make_float2(invG, invG);
     float2 xx = make_float2(0.0f, 0.0f), xg = make_float2(0.0f, 0.0f);
@@ -225,17 +231,16 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
       const int kk = (tg + b * tpr) < C.K ? tg + b * tpr : C.K - 1;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint4 gv4 = lds128(smem_u32(smem + ((size_t)j * C.K + kk) * 16));
-        const uint32_t gv[4] = {gv4.x, gv4.y, gv4.z, gv4.w};
+        float2 gf[4];
+        gamma_slot<true>(smem, C.K, j, kk, gf);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int w = 4 * j + i;
           const float2 x2 = bf16x2_to_f2(xr[b][w]);
-          const float2 d2 = bf16x2_to_f2(dr[b][w]);
-          const float2 g2 = mul2(bf16x2_to_f2(gv[i]), d2);
+          const float2 p2 = mul2(bf16x2_to_f2(dr[b][w]), x2);
           xx = fma2(x2, x2, xx);
-          xg = fma2(x2, g2, xg);
-          const float2 a2 = fma2(mul2(d2, x2), invG2, make_float2(acc[b][2 * w], acc[b][2 * w + 1]));
+          xg = fma2(p2, gf[i], xg);
+          const float2 a2 = fma2(p2, invG2, make_float2(acc[b][2 * w], acc[b][2 * w + 1]));
           acc[b][2 * w] = a2.x;
           acc[b][2 * w + 1] = a2.y;
         }
@@ -277,14 +282,14 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int kk = k < C.K ? k : C.K - 1;
-        const uint4 gv4 = lds128(smem_u32(smem + ((size_t)j * C.K + kk) * 16));
-        const uint32_t gv[4] = {gv4.x, gv4.y, gv4.z, gv4.w};
+        float2 gf[4];
+        gamma_slot<true>(smem, C.K, j, kk, gf);
         uint32_t o[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int w = 4 * j + i;
           const float2 x2 = bf16x2_to_f2_again(xr[b][w]);
-          const float2 g2 = mul2(bf16x2_to_f2_again(gv[i]), bf16x2_to_f2_again(dr[b][w]));
+          const float2 g2 = mul2(gf[i], bf16x2_to_f2_again(dr[b][w]));
           const float2 r = mul2(fma2(x2, ncoef2, g2), sdx2);
           const __nv_bfloat162 h = __floats2bfloat162_rn(r.x, r.y);
           o[i] = *reinterpret_cast<const uint32_t*>(&h);
@@ -367,16 +372,28 @@ __global__ void __launch_bounds__(bwd_max_threads(BPT), 1) row_bwd_kernel(const 
 
 // dgamma[j] = sum over the n_part partial rows, in a fixed order: thread
 // (tx, ty) of a 32 x 32 CTA adds rows ty, ty + 32, ... of column j = 32 *
-// blockIdx.x + tx; the 32 lane sums are then added in ty order.
+// blockIdx.x + tx (eight rows' loads in flight at a time, added in row
+// order); the 32 lane sums are then added in ty order.
 __global__ void __launch_bounds__(1024) dgamma_reduce_kernel(const float* partial, int64_t n_part,
                                                              int D, uint16_t* dgamma) {
   __shared__ float sh[32][33];
   griddep_wait();                  // the backward kernel's partial rows are complete
+  griddep_launch_dependents();     // the next kernel may start its set-up
   const int tx = threadIdx.x, ty = threadIdx.y;
   const int j = blockIdx.x * 32 + tx;
   float s = 0.0f;
-  if (j < D)
-    for (int64_t r = ty; r < n_part; r += 32) s += partial[r * D + j];
+  if (j < D) {
+    for (int64_t r0 = ty; r0 < n_part; r0 += 8 * 32) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t r = r0 + 32 * u;
+        v[u] = r < n_part ? partial[r * D + j] : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s += v[u];
+    }
+  }
   sh[ty][tx] = s;
   __syncthreads();
   if (ty == 0 && j < D) {
