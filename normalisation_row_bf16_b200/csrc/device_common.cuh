@@ -263,6 +263,13 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 
 __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) { return make_float2(bf16lo(w), bf16hi(w)); }
 
+// min(a, |b|, |c|) (a NaN operand is ignored).
+__device__ __forceinline__ float min3_abs(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+  return d;
+}
+
 // max(a, |b|, |c|), propagating NaN.
 __device__ __forceinline__ float max3_abs_nan(float a, float b, float c) {
   float d;
@@ -444,10 +451,22 @@ __device__ __forceinline__ void philox4x32_10_x2(uint4& a, uint4& b, const Philo
 // into the kept mantissa exactly when v rounds up (the carry may step into the
 // next binade, which is lo + step; it cannot reach the sign, |v| <= 448), and
 // clearing the 20 low bits leaves the grid value with v's sign.
+//
+// Split for speed: sr_e4m3_grid_fast is the integer form, exact for |v| >=
+// 2^-6 and for zero; sr_e4m3_small_key(b) is below kSrE4m3SmallKey exactly
+// when 0 < |v| < 2^-6 (zero and the sign map out of range).  A caller takes
+// the integer form everywhere and redoes with sr_e4m3_grid only the elements
+// the key flags, once a cheap test (the minimum magnitude) finds any.
+__device__ __forceinline__ float sr_e4m3_grid_fast(uint32_t b, uint32_t r) {
+  return __uint_as_float((b + ((~r) >> 12)) & 0xFFF00000u);
+}
+constexpr uint32_t kSrE4m3SmallKey = 2u * 0x3C800000u - 2u;
+__device__ __forceinline__ uint32_t sr_e4m3_small_key(uint32_t b) { return b + b - 2u; }
+
 __device__ __forceinline__ float sr_e4m3_grid(float v, uint32_t r) {
   const uint32_t b = __float_as_uint(v);
   const uint32_t ab = b & 0x7FFFFFFFu;
-  if (ab >= 0x3C800000u) return __uint_as_float((b + ((~r) >> 12)) & 0xFFF00000u);
+  if (ab >= 0x3C800000u) return sr_e4m3_grid_fast(b, r);
   const float a = __uint_as_float(ab);
   const float lo = truncf(a * 512.0f) * (1.0f / 512.0f);
   const uint32_t thr = __float2uint_ru((a - lo) * 2199023255552.0f);   // 2^41

@@ -441,15 +441,32 @@ __device__ __forceinline__ uint8_t quantise_block(const float (&y)[32], float a,
       uint4 rr[2] = {make_uint4((uint32_t)ctr, (uint32_t)(ctr >> 32), 0u, 0u),
                      make_uint4((uint32_t)(ctr + 1), (uint32_t)((ctr + 1) >> 32), 0u, 0u)};
       philox4x32_10_x2(rr[0], rr[1], pk);
+      // the slot's 8 values onto the grid by the integer form; magnitudes
+      // under 2^-6 (rare after the block scale) are redone exactly, behind a
+      // warp vote on the slot's minimum magnitude (zeros trip it too, and the
+      // key then picks out the nonzero ones) so that no element pays for that
+      // path otherwise
+      const uint32_t rw[8] = {rr[0].x, rr[0].y, rr[0].z, rr[0].w, rr[1].x, rr[1].y, rr[1].z, rr[1].w};
+      float v[8], gv[8];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint4 r = rr[h];
-        const int i0 = sl * 8 + h * 4;
-        const float2 v0 = mul2(make_float2(y[i0], y[i0 + 1]), inv2);
-        const float2 v1 = mul2(make_float2(y[i0 + 2], y[i0 + 3]), inv2);
-        qw[sl * 2 + h] = cvt_e4m3x4_rn(sr_e4m3_grid(v0.x, r.x), sr_e4m3_grid(v0.y, r.y),
-                                       sr_e4m3_grid(v1.x, r.z), sr_e4m3_grid(v1.y, r.w));
+      for (int i = 0; i < 4; ++i) {
+        const float2 t = mul2(make_float2(y[sl * 8 + 2 * i], y[sl * 8 + 2 * i + 1]), inv2);
+        v[2 * i] = t.x;
+        v[2 * i + 1] = t.y;
       }
+      float vmin = min3_abs(fabsf(v[0]), v[1], v[2]);
+      vmin = min3_abs(vmin, v[3], v[4]);
+      vmin = min3_abs(vmin, v[5], v[6]);
+      vmin = min3_abs(vmin, v[7], v[7]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) gv[i] = sr_e4m3_grid_fast(__float_as_uint(v[i]), rw[i]);
+      if (__any_sync(0xFFFFFFFFu, vmin < 0.015625f)) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (sr_e4m3_small_key(__float_as_uint(v[i])) < kSrE4m3SmallKey) gv[i] = sr_e4m3_grid(v[i], rw[i]);
+      }
+      qw[sl * 2] = cvt_e4m3x4_rn(gv[0], gv[1], gv[2], gv[3]);
+      qw[sl * 2 + 1] = cvt_e4m3x4_rn(gv[4], gv[5], gv[6], gv[7]);
     }
   }
   if constexpr (ELEM == kElemE4M3) {

@@ -97,6 +97,28 @@ def test_mxnorm_fwd_sr_ragged(T, D):
     check_mxnorm_fwd(xd, gd, 2.0, ops.SR, D, q, s, G)
 
 
+@pytest.mark.parametrize("D", [1024, 4096])
+def test_mxnorm_fwd_sr_small_magnitudes(D):
+    """Stochastic rounding where many scaled values fall under 2^-6 (the E4M3
+    subnormal steps, where the kernel leaves its integer fast form for the exact
+    threshold): each block holds one large value and others spread over 2^-30
+    .. 1 of it, with zeros mixed in."""
+    T = 96
+    gen = torch.Generator().manual_seed(D)
+    mag = torch.exp2(-30.0 * torch.rand(T, D, generator=gen))
+    sign = torch.where(torch.rand(T, D, generator=gen) < 0.5, -1.0, 1.0)
+    x = (sign * mag).view(T, D // 32, 32)
+    x[:, :, 0] = 4.0
+    x = x.view(T, D)
+    x[torch.rand(T, D, generator=gen) < 0.05] = 0.0
+    x = x.to(torch.bfloat16)
+    xd = _dev(x)
+    for seed in (1, 0xDEAD_BEEF_0123):
+        q, s, G = ops.mxnorm_fwd(xd, None, 2.0, rounding=ops.SR, seed=seed)
+        torch.cuda.synchronize()
+        check_mxnorm_fwd(xd, None, 2.0, ops.SR, seed, q, s, G)
+
+
 def test_mxnorm_fwd_special_rows():
     D = 1024
     x = torch.zeros(8, D, dtype=torch.bfloat16)
