@@ -367,6 +367,41 @@ __device__ __forceinline__ float nvfp4_scale_value(float a) {
   return fminf(s, 448.0f);
 }
 
+// Two E4M3 codes (bits 0..7 and 8..15) -> their exact values.
+__device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t cc) {
+  float lo, hi;
+  asm("{\n\t.reg .b16 c;\n\t.reg .b32 h2;\n\t.reg .f16 l, h;\n\t"
+      "cvt.u16.u32 c, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h2, c;\n\t"
+      "mov.b32 {l, h}, h2;\n\t"
+      "cvt.f32.f16 %0, l;\n\t"
+      "cvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(cc));
+  return make_float2(lo, hi);
+}
+
+// The NVFP4 scale codes of two 16-element halves with absmax a0, a1 (>= 0
+// finite): code 0 in bits 0..7, code 1 in bits 8..15 -- the codes of
+// nvfp4_scale_value.  The wanted code is the smallest with 6 * value >= a
+// (0x7E, 448, when none).  u = fl(a * c) is below a / 6 by under 2^-23 of it
+// (see there; for a tiny a, by under 2^-150 absolute), far less than any E4M3
+// step, so: with no grid value in [u, a / 6] the wanted code is u rounded up,
+// which is u's nearest-even code or the next; with one, g, u's nearest code
+// is g itself, and the wanted code is g (a = 6 g) or the next.  So take the
+// nearest-even codes of both halves in one packed conversion (saturating at
+// 448) and step each up once where 6 * value < a, never past 0x7E.  6 * value
+// is exact in fp32.
+__device__ __forceinline__ uint32_t nvfp4_scale_codes2(float a0, float a1) {
+  constexpr float kC6 = 0.16666665673255920f;
+  const float2 u = mul2(make_float2(a0, a1), make_float2(kC6, kC6));
+  uint32_t cc = cvt_e4m3x2_rn(u.x, u.y);
+  const float2 six = mul2(e4m3x2_to_f2(cc), make_float2(6.0f, 6.0f));
+  const uint32_t up0 = (six.x < a0 && (cc & 0xFFu) != 0x7Eu) ? 1u : 0u;
+  const uint32_t up1 = (six.y < a1 && (cc >> 8) != 0x7Eu) ? 0x100u : 0u;
+  return cc + up0 + up1;
+}
+
 // E4M3 code of an E4M3 value v >= 0 held exactly in fp32: (E - 127 + 7) << 3 |
 // mantissa from 2^-6 up; below, v = k * 2^-9 with k = 0..7, read off the bits
 // of v * 512 + 2^23.

@@ -550,10 +550,12 @@ __device__ __forceinline__ uint32_t quantise_nvfp4(const float (&y)[32], const f
   ah[1] = max3_abs_nan(sm[2], sm[3], 0.0f);
   uint32_t code[2], and_mask[2], or_mask[2];
   float inv[2];
+  const bool bad2[2] = {!(ah[0] <= 3.402823466e38f), !(ah[1] <= 3.402823466e38f)};   // NaN or infinity
+  const uint32_t cc = nvfp4_scale_codes2(bad2[0] ? 0.0f : ah[0], bad2[1] ? 0.0f : ah[1]);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const bool bad = !(ah[h] <= 3.402823466e38f);                  // NaN or infinity
-    code[h] = bad ? 0x7Fu : e4m3_code_of(nvfp4_scale_value(ah[h]));
+    const bool bad = bad2[h];
+    code[h] = bad ? 0x7Fu : (h == 0 ? (cc & 0xFFu) : (cc >> 8));
     inv[h] = rtab[code[h]];                                        // 0 for codes 0 and 0x7F
     // a bad half's codes are all 0x7; a zero scale's are 0 (not -0)
     and_mask[h] = bad ? 0u : (code[h] == 0 ? 0u : 0xFFFFFFFFu);
