@@ -763,7 +763,9 @@ def run_gemm_leg(args, w, rank, world, dev, barrier):
             "roofline": {"bound": "tensor", "achieved": round(tflops / world, 1), "peak": round(fp8_peak, 1),
                          "unit": "TFLOP/s", "frac": round(tflops / world / fp8_peak, 4),
                          "peak_source": f"{src} bf16 x 2 (nominal fp8/bf16 ratio)"},
-            "kernel": "gemm_mxfp8_kernel (tcgen05 mxf8f6f4 block_scale, 128x256 tiles)"}
+            "kernel": ("gemm_mxfp8_wide_kernel (tcgen05 mxf8f6f4 block_scale, 256x192 tiles)"
+                       if T % 256 == 0 and N % 384 == 0 else
+                       "gemm_mxfp8_kernel (tcgen05 mxf8f6f4 block_scale, 128x256 tiles)")}
 
 
 def nvfp4_bytes(T, D):

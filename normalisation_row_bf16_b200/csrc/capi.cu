@@ -794,8 +794,8 @@ int mxnorm_set_tuning(int consumer_threads, int stages, int ctas_per_sm) {
 
 int mxnorm_set_gemm_tiles(int mode) {
   t_err.clear();
-  if (mode != 0 && mode != 1) return fail(MXN_ERR_ARG, "gemm tile mode = %d", mode);
-  gemm_mxfp8_set_pairs(mode);
+  if (mode < 0 || mode > 2) return fail(MXN_ERR_ARG, "gemm tile mode = %d", mode);
+  gemm_mxfp8_set_tiles(mode);
   return MXN_OK;
 }
 

@@ -6,8 +6,11 @@
 //   C[m, n] = sum_k A(m, k) * B(n, k),  A(m,k) = e4m3(a_q[m,k]) * 2^(a_s[m,k/32] - 127),
 //   B likewise, fp32 accumulation in tensor memory, bf16 output.
 //
-// Persistent CTAs, one per SM, walk the 128 x 256 output tiles (tile t, then
-// t + gridDim.x, ...; M-tiles fastest, so the CTAs in flight share B tiles):
+// Three tile shapes (gemm_mxfp8_set_tiles): 256 x 192 by default where the
+// shape allows (described with its kernel below), 128 x 256 otherwise, and
+// 256 x 256 on CTA pairs on request.  The 128 x 256 kernel: persistent CTAs,
+// one per SM, walk the output tiles (tile t, then t + gridDim.x, ...; M-tiles
+// fastest, so the CTAs in flight share B tiles):
 //  * warp 0, one thread: the producer streams 128-element K stages of A
 //    (128 x 128 B) and B (256 x 128 B) into a 4-stage shared-memory ring with
 //    TMA tensor copies (128-byte swizzle, no multicast), and the stage's scale
@@ -37,13 +40,15 @@
 
 namespace mxn {
 
-// Process-wide switch of the tile shape (mxnorm_set_gemm_tiles).  Single-CTA
-// tiles by default: the pair kernel moves a third fewer operand bytes from L2
-// but measured slower on B200 (8192 x 6144 x 4096: 193 against 177 us under
-// ncu, tensor pipe active 52% against 57%).
-static int g_gemm_pairs = 0;
-void gemm_mxfp8_set_pairs(int on) { g_gemm_pairs = on ? 1 : 0; }
-static bool gemm_pair_enabled() { return g_gemm_pairs != 0; }
+// Process-wide switch of the tile shape (mxnorm_set_gemm_tiles): 0 (default)
+// = 256 x 192 single-CTA tiles where M % 256 == 0 and N % 384 == 0, else 128 x
+// 256; 1 = 256 x 256 tiles on CTA pairs where M % 256 == 0; 2 = 128 x 256
+// single-CTA tiles.  Measured on B200 at 8192 x 6144 x 4096 (20-launch graphs,
+// interleaved, median): 179 us for 256 x 192, 193 us for 128 x 256 and 216 us
+// for the pairs, which move a third fewer operand bytes from L2 than 128 x 256
+// but stall on the pair's coupling.
+static int g_gemm_tiles = 0;
+void gemm_mxfp8_set_tiles(int mode) { g_gemm_tiles = mode; }
 
 namespace {
 
@@ -72,7 +77,7 @@ struct Smem {
   uint64_t mma_done;                             // every MMA of this CTA retired
   uint32_t tmem_base;
   uint32_t failed;
-  uint8_t cstage[kEpiWarps][32 * 64];            // per epilogue warp: 32 rows x 32 bf16 of C
+  alignas(128) uint8_t cstage[kEpiWarps][32 * 64];            // per epilogue warp: 32 rows x 32 bf16 of C
 };
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -387,7 +392,7 @@ struct Smem2 {
   uint64_t mma_done;                                         // CTA 0's
   uint32_t tmem_base;
   uint32_t failed;
-  uint8_t cstage[kEpiWarps][32 * 64];
+  alignas(128) uint8_t cstage[kEpiWarps][32 * 64];
 };
 
 __device__ __forceinline__ bool failed_flag2(const Smem2& S) {
@@ -664,6 +669,273 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 
+// ------------------------------------------------------------------ 256 x 192 tiles
+//
+// One CTA per SM on 256 x 192 output tiles: two M = 128 accumulators of 192
+// columns each (384 of the 512 tensor-memory columns; the scales of 3 stages
+// take 48 more), so each K stage's operands -- A 256 x 128 B, B 192 x 128 B --
+// feed twice the MMA work of a 128 x 256 tile's 48 KiB for 56 KiB: 22% fewer
+// bytes per flop from L2, which bounds the 128 x 256 kernel, and 8192 x 6144
+// splits into 1024 tiles (6.9 per SM) instead of 1536 (10.4).  Needs M % 256
+// == 0 and N % 384 == 0 (every tile's B rows then lie in two whole 128-row
+// scale atoms).
+//  * warp 0, one thread: TMA tensor copies of A (box 128 B x 256 rows) and B
+//    (128 B x 192 rows) and bulk copies of the two A scale atoms and of the two
+//    B atoms that cover the tile's 192 rows;
+//  * warp 2, running ahead of the MMA thread: rebuilds each stage's B scales
+//    in tile order (an odd N-tile starts 64 rows into its first atom: lane l's
+//    16 bytes hold its 4 row groups, so the tile's rows 0..127 are groups 2, 3
+//    of the first atom and 0, 1 of the second) and signals the stage ready --
+//    on the MMA thread's path this cost every stage a few hundred cycles;
+//  * warp 1, one thread: copies the four scale atoms into tensor memory and
+//    issues, for each 32-element K step, one MMA (M 128, N 192) per
+//    accumulator;
+//  * warps 3..14: lane quarter (warp % 4) x 128 of the 384 accumulator
+//    columns each, read, handed back, converted and stored as in the
+//    128 x 256 kernel.
+constexpr int kWM = 256, kWN = 192;
+constexpr int kWStages = 3;
+constexpr int kWEpiWarps = 12;
+constexpr int kWThreads = 96 + 32 * kWEpiWarps;  // producer, MMA, scale warp, epilogue warps
+constexpr uint32_t kWABytes = kWM * kTileK;     // 32 KiB
+constexpr uint32_t kWBBytes = kWN * kTileK;     // 24 KiB
+constexpr uint32_t kWStageTx = kWABytes + kWBBytes + 4 * kSfaBytes;
+constexpr uint32_t kWSfCol0 = 384;              // scales: 16 columns per stage
+
+struct SmemW {
+  uint8_t a[kWStages][kWABytes];                // 1024-aligned (128B swizzle atoms)
+  uint8_t b[kWStages][kWBBytes];
+  uint8_t sfa[kWStages][2 * kSfaBytes];         // A rows 0..127, 128..255 of the tile
+  uint8_t sfb[kWStages][2 * kSfaBytes];         // the two B atoms covering the tile, as stored
+  uint8_t sfb_t[kWStages][2 * kSfaBytes];       // B rows 0..127, 128..191 (+ zero groups) of the tile
+  uint64_t full[kWStages];
+  uint64_t empty[kWStages];
+  uint64_t sf_ready[kWStages];                  // scale warp -> MMA: the stage's B scales rebuilt
+  uint64_t acc_full;
+  uint64_t acc_empty;
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  uint32_t failed;
+  alignas(128) uint8_t cstage[kWEpiWarps][32 * 64];
+};
+
+__device__ __forceinline__ uint32_t instr_desc_n(uint32_t sf_id, uint32_t n) {
+  return (sf_id << 4) | ((n >> 3) << 17) | (1u << 23) | ((uint32_t)(kTileM >> 4) << 24) | (sf_id << 29);
+}
+
+__device__ __forceinline__ bool failed_flag_w(const SmemW& S) {
+  return *reinterpret_cast<const volatile uint32_t*>(&S.failed) != 0;
+}
+
+__global__ void __launch_bounds__(kWThreads, 1)
+    gemm_mxfp8_wide_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                           const uint8_t* __restrict__ a_s, const uint8_t* __restrict__ b_s,
+                           uint16_t* __restrict__ c, int M, int N, int K, unsigned* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  SmemW& S = *reinterpret_cast<SmemW*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = M / kWM;
+  const int n_tiles_all = m_tiles * (N / kWN);
+  const int n_k = K / kTileK;
+  const int kp4 = K / 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kWStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+      mbar_init(&S.sf_ready[s], 1);
+    }
+    mbar_init(&S.acc_full, 1);
+    mbar_init(&S.acc_empty, kWEpiWarps);
+    mbar_init(&S.mma_done, 1);
+    S.failed = 0;
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  griddep_wait();
+  griddep_launch_dependents();
+
+  uint32_t n_issued = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- producer
+      uint32_t g = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles_all && ok; t += gridDim.x) {
+        const int mt = t % m_tiles, nt = t / m_tiles;
+        const int fa = (3 * nt) >> 1;            // first B scale atom of the tile's rows
+        for (int kb = 0; kb < n_k; ++kb, ++g) {
+          const int s = (int)(g % kWStages);
+          const uint32_t ph = (g / kWStages) & 1u;
+          if (!mbar_wait_bounded(&S.empty[s], ph ^ 1u, status) || failed_flag_w(S)) {
+            atomicOr(&S.failed, 1u);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&S.full[s], kWStageTx);
+          tma_load_2d(S.a[s], &map_a, kb * kTileK, mt * kWM, &S.full[s]);
+          tma_load_2d(S.b[s], &map_b, kb * kTileK, nt * kWN, &S.full[s]);
+          bulk_g2s_plain(S.sfa[s], a_s + ((size_t)(2 * mt) * (kp4 / 4) + kb) * 512, 512, &S.full[s]);
+          bulk_g2s_plain(S.sfa[s] + 512, a_s + ((size_t)(2 * mt + 1) * (kp4 / 4) + kb) * 512, 512, &S.full[s]);
+          bulk_g2s_plain(S.sfb[s], b_s + ((size_t)fa * (kp4 / 4) + kb) * 512, 512, &S.full[s]);
+          bulk_g2s_plain(S.sfb[s] + 512, b_s + ((size_t)(fa + 1) * (kp4 / 4) + kb) * 512, 512, &S.full[s]);
+          n_issued = g + 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------- MMA
+      uint32_t g = 0, it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles_all && ok; t += gridDim.x, ++it) {
+        if (!mbar_wait_bounded(&S.acc_empty, (it & 1u) ^ 1u, status) || failed_flag_w(S)) {
+          atomicOr(&S.failed, 1u);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < n_k; ++kb, ++g) {
+          const int s = (int)(g % kWStages);
+          const uint32_t ph = (g / kWStages) & 1u;
+          if (!mbar_wait_bounded(&S.full[s], ph, status) || !mbar_wait_bounded(&S.sf_ready[s], ph, status) ||
+              failed_flag_w(S)) {
+            atomicOr(&S.failed, 1u);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa_col = kWSfCol0 + (uint32_t)s * 16u, sfb_col = sfa_col + 8u;
+          tmem_cp_sf(tmem + sfa_col, smem_desc(smem_u32(S.sfa[s]), 0, 128, 0));
+          tmem_cp_sf(tmem + sfa_col + 4u, smem_desc(smem_u32(S.sfa[s] + 512), 0, 128, 0));
+          tmem_cp_sf(tmem + sfb_col, smem_desc(smem_u32(S.sfb_t[s]), 0, 128, 0));
+          tmem_cp_sf(tmem + sfb_col + 4u, smem_desc(smem_u32(S.sfb_t[s] + 512), 0, 128, 0));
+          const uint32_t a_base = smem_u32(S.a[s]), b_base = smem_u32(S.b[s]);
+#pragma unroll
+          for (int k = 0; k < kTileK / 32; ++k) {
+            const uint64_t bd = smem_desc(b_base + 32u * k, 16, 1024, 2);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t ad = smem_desc(a_base + (uint32_t)h * (kWABytes / 2) + 32u * k, 16, 1024, 2);
+              mma_mxf8(tmem + (uint32_t)(h * kWN), ad, bd, instr_desc_n((uint32_t)k, kWN),
+                       (tmem + sfa_col + 4u * h) | ((uint32_t)k << 30), (tmem + sfb_col) | ((uint32_t)k << 30),
+                       (kb > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit(&S.empty[s]);
+        }
+        if (ok) tc_commit(&S.acc_full);
+      }
+      tc_commit(&S.mma_done);
+      if (!ok) tc_commit(&S.acc_full);
+    }
+  } else if (warp == 2) {
+    // ----------------------------------------------------- B scale rebuild
+    // Runs ahead of the MMA thread (see above for the row-group order).
+    uint32_t g = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles_all && ok; t += gridDim.x) {
+      const bool odd = ((t / m_tiles) & 1) != 0;
+      for (int kb = 0; kb < n_k; ++kb, ++g) {
+        const int s = (int)(g % kWStages);
+        const uint32_t ph = (g / kWStages) & 1u;
+        const bool w = mbar_wait_bounded(&S.full[s], ph, status) && !failed_flag_w(S);
+        if (!__all_sync(0xFFFFFFFFu, w)) {
+          if (lane == 0) atomicOr(&S.failed, 1u);
+          ok = false;
+          break;
+        }
+        const uint4 a0 = reinterpret_cast<const uint4*>(S.sfb[s])[lane];
+        const uint4 a1 = reinterpret_cast<const uint4*>(S.sfb[s] + 512)[lane];
+        const uint4 t0 = odd ? make_uint4(a0.z, a0.w, a1.x, a1.y) : a0;
+        const uint4 t1 = odd ? make_uint4(a1.z, a1.w, 0u, 0u) : make_uint4(a1.x, a1.y, 0u, 0u);
+        reinterpret_cast<uint4*>(S.sfb_t[s])[lane] = t0;
+        reinterpret_cast<uint4*>(S.sfb_t[s] + 512)[lane] = t1;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.sf_ready[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 3;
+    const int quarter = warp & 3;
+    const int third = e >> 2;                    // accumulator columns 128 * third ..
+    uint32_t it = 0;
+    for (int t = blockIdx.x; t < n_tiles_all; t += gridDim.x, ++it) {
+      const int mt = t % m_tiles, nt = t / m_tiles;
+      const bool got = mbar_wait_bounded(&S.acc_full, it & 1u, status);
+      tc_fence_after();
+      if (!got || failed_flag_w(S)) {
+        if (lane == 0) atomicOr(&S.failed, 1u);
+        break;
+      }
+      uint32_t r[4][32];
+      const uint32_t ta = tmem + (uint32_t)(third * 128) + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tmem_ld32(ta + 32u * j, r[j]);
+      tmem_ld_fence(r[0], true);
+#pragma unroll
+      for (int j = 1; j < 4; ++j) tmem_ld_fence(r[j], false);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.acc_empty);
+      uint8_t* stg = S.cstage[e];
+      const uint32_t stg_u32 = smem_u32(stg);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int col = third * 128 + 32 * j;    // of the 384: accumulator col / 192, column col % 192
+        const int acc = col >= kWN ? 1 : 0;
+        uint16_t* ctile = c + (size_t)(mt * kWM + acc * 128 + quarter * 32) * N + (size_t)nt * kWN + (col - acc * kWN);
+        uint32_t o[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(r[j][2 * i]), __uint_as_float(r[j][2 * i + 1]));
+          o[i] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t off = (uint32_t)lane * 64u + (uint32_t)((v ^ ((lane >> 1) & 3)) * 16);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg_u32 + off), "r"(o[4 * v]),
+                       "r"(o[4 * v + 1]), "r"(o[4 * v + 2]), "r"(o[4 * v + 3])
+                       : "memory");
+        }
+        __syncwarp();
+#pragma unroll
+        for (int t2 = 0; t2 < 4; ++t2) {
+          const int rr = t2 * 8 + (lane >> 2), cc = lane & 3;
+          const uint4 v4 = lds128(stg_u32 + (uint32_t)rr * 64u + (uint32_t)((cc ^ ((rr >> 1) & 3)) * 16));
+          *reinterpret_cast<uint4*>(ctile + (size_t)rr * N + 8 * cc) = v4;
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1 && lane == 0) mbar_wait_bounded(&S.mma_done, 0, status);
+  if (warp == 0 && lane == 0 && failed_flag_w(S))
+    for (uint32_t j = (n_issued > (uint32_t)kWStages ? n_issued - kWStages : 0); j < n_issued; ++j)
+      mbar_wait_bounded(&S.full[j % kWStages], (j / kWStages) & 1u, status);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -733,6 +1005,36 @@ int pair_clusters(int dev) {
   return n;
 }
 
+int launch_wide(const void* a_q, const void* a_s, const void* b_q, const void* b_s, void* c, int M, int N, int K,
+                int sms, unsigned* status, cudaStream_t stream, const char** why) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, a_q, M, K, kWM) || !make_map(&mb, b_q, N, K, kWN)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return -1;
+  }
+  const size_t smem = sizeof(SmemW);
+  cudaError_t e = cudaFuncSetAttribute(gemm_mxfp8_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) { *why = cudaGetErrorString(e); return (int)e; }
+  const int tiles = (M / kWM) * (N / kWN);
+  const uint8_t* as = static_cast<const uint8_t*>(a_s);
+  const uint8_t* bs = static_cast<const uint8_t*>(b_s);
+  uint16_t* cp = static_cast<uint16_t*>(c);
+  void* argv[] = {&ma, &mb, &as, &bs, &cp, &M, &N, &K, &status};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tiles < sms ? tiles : sms);
+  cfg.blockDim = dim3(kWThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelExC(&cfg, (const void*)gemm_mxfp8_wide_kernel, argv);
+  if (e != cudaSuccess) { *why = cudaGetErrorString(e); return (int)e; }
+  return 0;
+}
+
 int launch_pair(const void* a_q, const void* a_s, const void* b_q, const void* b_s, void* c, int M, int N, int K,
                 int clusters, unsigned* status, cudaStream_t stream, const char** why) {
   CUtensorMap ma, mb, msa, msb;
@@ -771,8 +1073,11 @@ size_t gemm_mxfp8_smem_bytes() { return sizeof(Smem) + 1024; }
 // Launch: returns 0, or -1 (tensor map could not be encoded) / cuda error code.
 int gemm_mxfp8_launch(const void* a_q, const void* a_s, const void* b_q, const void* b_s, void* c, int M,
                       int N, int K, int sms, unsigned* status, cudaStream_t stream, const char** why) {
+  // 256 x 192 tiles by default where the shape allows.
+  if (g_gemm_tiles == 0 && M % kWM == 0 && N % (2 * kWN) == 0)
+    return launch_wide(a_q, a_s, b_q, b_s, c, M, N, K, sms, status, stream, why);
   // 256 x 256 tiles on CTA pairs where the shape allows and the device has room.
-  if (M % 256 == 0 && N % 256 == 0 && gemm_pair_enabled()) {
+  if (M % 256 == 0 && N % 256 == 0 && g_gemm_tiles == 1) {
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) {
       const int ncl = pair_clusters(dev);

@@ -304,7 +304,8 @@ def set_tuning(consumer_threads: int = 0, stages: int = 0, ctas_per_sm: int = 0)
 
 
 def set_gemm_tiles(mode: int = 0):
-    """0: single-CTA 128 x 256 GEMM tiles (default); 1: CTA-pair 256 x 256 tiles where M % 256 == 0."""
+    """0 (default): single-CTA 256 x 192 GEMM tiles where M % 256 == 0 and N % 384 == 0, else 128 x 256;
+    1: CTA-pair 256 x 256 tiles where M % 256 == 0; 2: single-CTA 128 x 256 tiles."""
     _check(lib().mxnorm_set_gemm_tiles(int(mode)))
 
 

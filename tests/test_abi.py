@@ -108,7 +108,8 @@ def test_tuning_validation(L):
     assert L.mxnorm_set_tuning(0, 0, 9) == ops.MXN_ERR_ARG
     assert L.mxnorm_set_tuning(256, 4, 2) == ops.MXN_OK
     assert L.mxnorm_set_tuning(0, 0, 0) == ops.MXN_OK
-    assert L.mxnorm_set_gemm_tiles(2) == ops.MXN_ERR_ARG
+    assert L.mxnorm_set_gemm_tiles(3) == ops.MXN_ERR_ARG
+    assert L.mxnorm_set_gemm_tiles(2) == ops.MXN_OK
     assert L.mxnorm_set_gemm_tiles(-1) == ops.MXN_ERR_ARG
     assert L.mxnorm_set_gemm_tiles(1) == ops.MXN_OK
     assert L.mxnorm_set_gemm_tiles(0) == ops.MXN_OK

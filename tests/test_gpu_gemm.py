@@ -105,9 +105,10 @@ def test_gemm_pair_tiles_match_single_cta_tiles(M, N, K):
     in the same order per output, so the outputs are identical; the pair
     kernel's result is also checked against the oracle on sampled entries."""
     aq, a_s_mma, a_s, bq, b_s_mma, b_s = _operands(M, N, K, seed=M + N)
-    c_single = ops.mxfp8_gemm(aq, a_s_mma, bq, b_s_mma, M, N, K)
-    ops.set_gemm_tiles(1)
+    ops.set_gemm_tiles(2)
     try:
+        c_single = ops.mxfp8_gemm(aq, a_s_mma, bq, b_s_mma, M, N, K)
+        ops.set_gemm_tiles(1)
         c_pair = ops.mxfp8_gemm(aq, a_s_mma, bq, b_s_mma, M, N, K)
     finally:
         ops.set_gemm_tiles(0)
@@ -117,3 +118,28 @@ def test_gemm_pair_tiles_match_single_cta_tiles(M, N, K):
     ii = np.concatenate([rng.integers(0, M, 256), [0, M - 1, 127, 128, 255]])
     jj = np.concatenate([rng.integers(0, N, 256), [0, N - 1, 127, 128, 255]])
     _check(aq, a_s, bq, b_s, c_pair, ii, jj)
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 768, 128), (512, 1536, 256), (2048, 1536, 1024), (8192, 6144, 4096)])
+def test_gemm_wide_tiles_match_128x256_tiles(M, N, K):
+    """The default 256 x 192 tiles (these shapes have M % 256 == 0 and N % 384
+    == 0): odd N-tiles start 64 rows into a 128-row scale atom, which the
+    kernel rebuilds in tile order; the outputs must equal the 128 x 256
+    kernel's (set_gemm_tiles(2)), and sampled entries the oracle's (including
+    both sides of every atom and tile boundary)."""
+    aq, a_s_mma, a_s, bq, b_s_mma, b_s = _operands(M, N, K, seed=M + 3 * N)
+    c_wide = ops.mxfp8_gemm(aq, a_s_mma, bq, b_s_mma, M, N, K)
+    ops.set_gemm_tiles(2)
+    try:
+        c_single = ops.mxfp8_gemm(aq, a_s_mma, bq, b_s_mma, M, N, K)
+    finally:
+        ops.set_gemm_tiles(0)
+    torch.cuda.synchronize()
+    assert torch.equal(c_wide, c_single)
+    rng = np.random.default_rng(M + 2)
+    edges = [0, 63, 64, 127, 128, 191, 192, 255, 256, 383]
+    ii = np.concatenate([rng.integers(0, M, 256), [e % M for e in edges], [M - 1]])
+    jj = np.concatenate([rng.integers(0, N, 256), [e % N for e in edges], [N - 1]])
+    jj = np.concatenate([jj, [e % N for e in edges]])
+    ii = np.concatenate([ii, [(M - 1 - e) % M for e in edges]])
+    _check(aq, a_s, bq, b_s, c_wide, ii, jj)
