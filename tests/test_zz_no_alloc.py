@@ -48,8 +48,12 @@ def test_noalloc_backward_matches_workspace_backward(T, D):
         dx_ref, dg_ref = ops.mxnorm_bwd(x, dy, g, G)
         dx = torch.full_like(x, float("nan"))
         dg = torch.full((D,), float("nan"), dtype=torch.bfloat16, device="cuda")
+        torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info()[0]
         _call_noalloc(x, dy, g, G, dx, dg)
         torch.cuda.synchronize()
+        if call == 1:   # the first call looked up the scratch array; later ones allocate nothing
+            assert torch.cuda.mem_get_info()[0] == free_before
         assert torch.equal(dx, dx_ref)
         assert rel_l2(dg.float().cpu().numpy(), dg_ref.float().cpu().numpy()) <= BWD_RTOL_L2
         assert torch.isfinite(dg.float()).all()
