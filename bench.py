@@ -412,8 +412,12 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step, s
 
     # end to end through the C ABI with pinned host buffers: the batch in row
     # chunks through three streams, so each chunk's host -> device copy, the
-    # MXNorm call and its device -> host copies overlap the neighbours'
-    # (rows are independent; nearest-even results do not depend on the chunking)
+    # MXNorm call and its device -> host copies overlap the neighbours' (rows
+    # are independent; nearest-even results do not depend on the chunking).
+    # Consecutive steps overlap too: a chunk's copy in waits only for the
+    # previous step's kernel on that chunk (its input buffer), and the kernel
+    # only for the previous step's copies out of that chunk (its outputs), so
+    # one step's copies out share the link's time with the next step's copies in.
     xh = xs[0].cpu().pin_memory()
     qh = torch.empty(T, D, dtype=torch.uint8).pin_memory()
     sh = torch.empty(T, D // 32, dtype=torch.uint8).pin_memory()
@@ -427,17 +431,23 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step, s
     s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev_in = [torch.cuda.Event() for _ in range(n_chunks)]
     ev_run = [torch.cuda.Event() for _ in range(n_chunks)]
+    ev_out = [torch.cuda.Event() for _ in range(n_chunks)]
     main = torch.cuda.current_stream()
 
-    def step_e2e():
-        s_in.wait_stream(main)
-        s_out.wait_stream(main)
+    def step_e2e(first):
+        if first:                      # start after everything queued on the main stream
+            for st in (s_in, s_run, s_out):
+                st.wait_stream(main)
         for c in range(n_chunks):
             r0, r1 = c * rows, (c + 1) * rows
+            if not first:
+                s_in.wait_event(ev_run[c])      # the previous step's kernel has read xd[c]
             with torch.cuda.stream(s_in):
                 xd[r0:r1].copy_(xh[r0:r1], non_blocking=True)
                 ev_in[c].record(s_in)
             s_run.wait_event(ev_in[c])
+            if not first:
+                s_run.wait_event(ev_out[c])     # the previous step's outputs of chunk c are on the host
             with torch.cuda.stream(s_run):
                 ops.mxnorm_fwd(xd[r0:r1], g, p, q=qd[r0:r1], scales=sd[r0:r1], G=Gd[r0:r1], stream=s_run)
                 ev_run[c].record(s_run)
@@ -446,16 +456,21 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step, s
                 qh[r0:r1].copy_(qd[r0:r1], non_blocking=True)
                 sh[r0:r1].copy_(sd[r0:r1], non_blocking=True)
                 Gh[r0:r1].copy_(Gd[r0:r1], non_blocking=True)
-        main.wait_stream(s_out)
-        main.wait_stream(s_run)
+                ev_out[c].record(s_out)
+
+    def join():
+        for st in (s_in, s_run, s_out):
+            main.wait_stream(st)
 
     Ke = min(args.steps, 100)
-    for _ in range(3):
-        step_e2e()
+    for i in range(3):
+        step_e2e(i == 0)
+    join()
     barrier()
     t0.record()
-    for _ in range(Ke):
-        step_e2e()
+    for i in range(Ke):
+        step_e2e(i == 0)
+    join()
     t1.record()
     barrier()
     te = torch.tensor([t0.elapsed_time(t1) / Ke], dtype=torch.float64, device=dev)
@@ -466,7 +481,7 @@ def run_extras(args, w, rank, world, dev, xs, g, n_sets, barrier, ms_per_step, s
                   "unit": "GB/s", "h2d_bytes_per_step": T * D * 2,
                   "d2h_bytes_per_step": T * D + T * (D // 32) + 4 * T,
                   "steps": Ke, "ms_per_step": round(te_ms, 4),
-                  "pipeline": f"{n_chunks} row chunks over 3 streams (copy in, MXNorm, copy out)"}
+                  "pipeline": f"{n_chunks} row chunks over 3 streams (copy in, MXNorm, copy out), consecutive steps overlapped"}
     # the check a user would make: the pipelined host results equal one device call's
     torch.cuda.synchronize()
     q_ref, s_ref, G_ref = ops.mxnorm_fwd(xd, g, p)
