@@ -247,8 +247,8 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int
   // 512 threads there too (MXFP4 / NVFP4 at 16384 x 8192: 65.5 -> 57.8 and
   // 100.1 -> 85.6 us; at 8192 x 4096: 17.8 -> 17.4 and 27.2 -> 26.0 us).
   // Rows under 33 blocks, and stochastic rounding (bound by the Philox
-  // arithmetic, so it wants every warp the registers allow), keep the largest
-  // CTA with extra stages while 176 KB covers them.
+  // arithmetic), keep the largest CTA the kernel is compiled for
+  // (fwd_launch_threads) with extra stages while 176 KB covers them.
   const bool widest = bpt == 1 || sr;
   const bool fp4 = elem != kElemE4M3;
   const int def_threads = widest ? fwd_max_threads(bpt) : (bpt == 2 || C.tpr > 64 || fp4 ? 512 : 384);

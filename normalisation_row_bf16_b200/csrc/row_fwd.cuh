@@ -53,8 +53,11 @@ __host__ __device__ constexpr int fwd_max_threads(int bpt) { return bpt >= 4 ? 5
 // Threads per CTA a kernel is compiled for (its __launch_bounds__).  One-warp
 // rows of 65..128 blocks of E4M3 codes with nearest-even rounding launch 384
 // threads, and are compiled for 384: up to 168 registers a thread.
+// Stochastic rounding with two blocks a thread launches 512 (up to 128
+// registers: the Philox rounds keep more in flight; measured on B200 at
+// 8192 x 4096: 51.9 -> 50.0 us against 640, and 56.0 at 384).
 __host__ __device__ constexpr int fwd_launch_threads(int bpt, int tpr, bool sr, int elem) {
-  return (bpt >= 4 && tpr == 32 && !sr && elem == 0) ? 384 : fwd_max_threads(bpt);
+  return (bpt >= 4 && tpr == 32 && !sr && elem == 0) ? 384 : ((sr && bpt == 2) ? 512 : fwd_max_threads(bpt));
 }
 constexpr int kRedSlots = 16;  // warps per row group, at most
 
