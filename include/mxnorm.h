@@ -255,10 +255,9 @@ int mxfp8_gemm(const void* a_q, const void* a_s, const void* b_q, const void* b_
 
 /*
  * mxnorm_bwd without a workspace argument, for callers that cannot allocate
- * device memory when they call: code recorded into a CUDA graph whose memory
- * plan is fixed up front, plugins inside an engine that owns every allocation,
- * and real-time loops that must not call cudaMalloc.  The paper has no
- * counterpart; this is a deployment convenience.
+ * device memory when they call: plugins inside an engine that owns every
+ * allocation, and real-time loops that must not call cudaMalloc.  The paper
+ * has no counterpart; this is a deployment convenience.
  *
  * Same arguments, results and limits as mxnorm_bwd (D <= 16384), except that
  * the dgamma partial sums live in one 8 MiB scratch array inside this library
