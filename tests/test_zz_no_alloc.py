@@ -2,11 +2,10 @@
 
 It serves callers that cannot allocate device memory at call time (engines
 that own every allocation, real-time loops).  It must give the same dx and
-dgamma as
-mxnorm_bwd with a caller-provided workspace, within the backward's tolerance,
-on two calls in a row (the second call reuses the library's scratch array as
-the first left it).  This file runs last so that a failure here leaves every
-other test already run.
+dgamma as mxnorm_bwd with a caller-provided workspace, within the backward's
+tolerance, on two calls in a row (the second call reuses the library's
+scratch array as the first left it).  This file runs last so that a failure
+here leaves every other test already run.
 """
 import ctypes
 
