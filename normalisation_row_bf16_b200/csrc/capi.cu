@@ -263,7 +263,7 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int
   }
   // gamma in shared memory: fp32 for up to 64 threads per row (D <= 8192), else bf16
   C.gamma_bytes = gamma_smem ? (uint32_t)align_up((gamma_fp32(C.tpr) ? 4u : 2u) * (uint32_t)D, 128) : 0u;
-  const size_t per_group = (size_t)C.stages * C.stage_bytes;
+  size_t per_group = (size_t)C.stages * C.stage_bytes;
   // MXNorm and MXCast rows of several warps stage each row's codes in shared
   // memory and write them with one bulk copy (D bytes of E4M3, half that of
   // E2M1); see kFwdBulkStores.
@@ -272,8 +272,8 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int
   // Shared memory per group: its ring, its code staging buffer, its 2 * stages
   // barriers and its two reduction slot arrays; plus gamma and 16 bytes of
   // alignment once.
-  const size_t per_group_base = per_group + (size_t)2 * C.stages * sizeof(uint64_t) +
-                                (size_t)2 * kRedSlots * sizeof(float2);
+  size_t per_group_base = per_group + (size_t)2 * C.stages * sizeof(uint64_t) +
+                          (size_t)2 * kRedSlots * sizeof(float2);
   int ng;
   if (g_tuning.consumer_threads) {
     ng = g_tuning.consumer_threads / C.gthreads;
@@ -288,12 +288,29 @@ int plan_fwd(int mode, bool sr, bool gamma_smem, int elem, int64_t T, int D, int
   int ng_fit = (int)((smem_cap - fixed) / per_group_base);
   if (ng_fit < ng_max) ng_max = ng_fit;
   ng = ng < 1 ? 1 : (ng > ng_max ? ng_max : ng);
+  // Few rows for the device (full CTAs would not reach every SM): fewer row
+  // groups per CTA, at least 4, so that the rows spread over (nearly) every SM,
+  // and one stage, since each group then gets about one row.  Measured on
+  // B200: 256 x 1024 4.06 -> 2.52 us, 1024 x 1024 4.30 -> 2.91, 256 x 4096
+  // 5.87 -> 4.28, 1024 x 4096 6.44 -> 5.07; shapes that fill every SM as
+  // planned are unchanged.
+  const int64_t n_rb = (T + C.rps - 1) / C.rps;
+  if (!g_tuning.consumer_threads && !g_tuning.stages && (n_rb + ng - 1) / ng < sms) {
+    int64_t ng_small = (n_rb + sms - 1) / sms;
+    if (ng_small < 4) ng_small = 4;
+    if (ng_small < ng) {
+      ng = (int)ng_small;
+      C.stages = 1;
+      per_group = C.stage_bytes;
+      per_group_base = per_group + 2 * sizeof(uint64_t) + (size_t)2 * kRedSlots * sizeof(float2);
+    }
+  }
   // The staging buffers must not cost row groups: where they would, codes are
   // stored directly.
   if (C.ostage_bytes && fixed + (size_t)ng * (per_group_base + C.ostage_bytes) > smem_cap) C.ostage_bytes = 0;
   if (C.tpr > 32 && ng > 15) ng = 15;  // named barriers 1..15
   C.ng = ng;
-  C.n_row_blocks = (T + C.rps - 1) / C.rps;
+  C.n_row_blocks = n_rb;
   C.ring_off = C.gamma_bytes;
   C.out_off = (uint32_t)align_up(C.ring_off + (size_t)ng * per_group, 128);
   C.bar_off = (uint32_t)align_up(C.out_off + (size_t)ng * C.ostage_bytes, 16);
