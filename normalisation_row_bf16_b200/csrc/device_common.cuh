@@ -219,24 +219,6 @@ __device__ __forceinline__ uint4 ldg128_nc(const void* p) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// max(a, |b|) propagating NaN.
-__device__ __forceinline__ float max_abs_nan(float a, float b) {
-  float d;
-  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(fabsf(b)));
-  return d;
-}
-
-// Absolute maximum of 32 bf16 values held as 16 packed words, as fp32.  The
-// comparison runs on the magnitude bits (for non-negative floats the integer
-// order is the numeric order), so a NaN, whose magnitude bits exceed those of
-// every number, propagates.
-__device__ __forceinline__ uint32_t absmax_bits_bf16x2(const uint32_t* w, int n) {
-  uint32_t m = 0;
-#pragma unroll
-  for (int i = 0; i < n; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
-  return max(m & 0xFFFFu, m >> 16);
-}
-
 __device__ __forceinline__ float bf16bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
 
 // 2^n for an integer n in [-126, 127], built from its exponent field.
@@ -401,18 +383,6 @@ __device__ __forceinline__ uint32_t nvfp4_scale_codes2(float a0, float a1) {
   const uint32_t up1 = (six.y < a1 && (cc >> 8) != 0x7Eu) ? 0x100u : 0u;
   return cc + up0 + up1;
 }
-
-// E4M3 code of an E4M3 value v >= 0 held exactly in fp32: (E - 127 + 7) << 3 |
-// mantissa from 2^-6 up; below, v = k * 2^-9 with k = 0..7, read off the bits
-// of v * 512 + 2^23.
-__device__ __forceinline__ uint32_t e4m3_code_of(float v) {
-  const uint32_t b = __float_as_uint(v);
-  const uint32_t sub = __float_as_uint(fmaf(v, 512.0f, 8388608.0f)) - 0x4B000000u;
-  return b >= 0x3C800000u ? ((((b >> 23) - 120u) << 3) | ((b >> 20) & 7u)) : sub;
-}
-
-// The NVFP4 block scale as its E4M3 code.
-__device__ __forceinline__ uint32_t nvfp4_scale_code(float a) { return e4m3_code_of(nvfp4_scale_value(a)); }
 
 // ------------------------------------------------------------------ E2M1 cast
 

@@ -138,24 +138,10 @@ __device__ __forceinline__ double exp2_int_f64(int n) {
   return n < -1022 ? 0.0 : __longlong_as_double((long long)(n + 1023) << 52);
 }
 
-__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
-  uint32_t r;
-  asm("redux.sync.add.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
-  return r;
-}
-__device__ __forceinline__ uint32_t seg_sum_u32(uint32_t v, int width) {
-  for (int off = width >> 1; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-  return v;
-}
-
 __device__ __forceinline__ double seg_sum_f64(double v, int width) {
   for (int off = width >> 1; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
   return v;
 }
-
-// The bf16 biased exponent used as the terms' reference: that of the maximum's
-// bits, 1 for subnormals and zero.
-__device__ __forceinline__ int ref_exponent(uint32_t mb) { return max((int)(mb >> 7), 1); }
 
 // Exact p-mean sums for p = 1, 2 in fp32 pairs.  A term t = (m / 2^Ew)^p has
 // at most 16 significant bits and lies in [0, 4).  It splits exactly into hi,
@@ -520,11 +506,6 @@ __device__ __forceinline__ void half_absmax_bits(const uint32_t (&w)[16], uint32
   hB = a[1];
 }
 
-// NVFP4 quantisation of one 32-element block (two 16-element NVFP4 blocks)
-// held in slot order: per half, the E4M3 scale code (nvfp4_scale_code of the
-// half's absmax, 0x7F for a half holding NaN or infinity), then the E2M1
-// codes of fl32(y * fl32(1/s)); a zero scale gives zero codes, a NaN half
-// codes 0x7.  Returns the two scale codes (half 0 in bits 0..7).
 // Absmax of each 8-element slot of a block's y (slot order), NaN-propagating.
 __device__ __forceinline__ void slot_absmax(const float (&y)[32], float (&sm)[4]) {
 #pragma unroll
@@ -545,6 +526,11 @@ __device__ __forceinline__ float e4m3_value_of_code(uint32_t c) {
   return e == 0 ? (float)m * (1.0f / 512.0f) : __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
+// NVFP4 quantisation of one 32-element block (two 16-element NVFP4 blocks)
+// held in slot order: per half, the E4M3 scale code (nvfp4_scale_codes2 of
+// the half's absmax, 0x7F for a half holding NaN or infinity), then the E2M1
+// codes of fl32(y * fl32(1/s)); a zero scale gives zero codes, a NaN half
+// codes 0x7.  Returns the two scale codes (half 0 in bits 0..7).
 template <bool SR>
 __device__ __forceinline__ uint32_t quantise_nvfp4(const float (&y)[32], const float (&sm)[4], int rot,
                                                    uint64_t idx0, const PhiloxKeys& pk, const float* rtab,
